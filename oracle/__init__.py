@@ -1,0 +1,180 @@
+"""Plain CPU oracle for the I2_S ternary x int8 matmul -- TEST INFRASTRUCTURE.
+
+Only the test suite, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU
+baseline leg may import this package.  It wraps ``i2s_oracle.c`` (scalar C,
+built with ``-O2 -ffp-contract=off -fno-fast-math``) through ctypes and works
+on numpy arrays.  It shares no code with the CUDA library in
+``i2_mpgemm_b200``; neither imports the other.
+
+Each function follows one step of the method as the web pages describe it;
+the C file lists the pages (by title and section) and every reading taken
+where they are silent.  Parity status: every function is pinned by the
+``-m "not gpu"`` tests (worked example, closed forms, brute force, error
+bounds) except the AbsMean ternarization's choice of eps and tie rule, which
+the pages leave open.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "i2s_oracle.c")
+_LIB = os.path.join(_HERE, "libi2s_oracle.so")
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-fPIC", "-shared"]
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (idempotent)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            i64, vp, f32, f64 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_double
+            lib.i2s_oracle_packed_bytes.restype = ctypes.c_size_t
+            lib.i2s_oracle_packed_bytes.argtypes = [i64, i64]
+            lib.i2s_oracle_pack.argtypes = [vp, i64, i64, vp]
+            lib.i2s_oracle_scale.restype = f32
+            lib.i2s_oracle_scale.argtypes = [vp, i64, i64]
+            lib.i2s_oracle_unpack.argtypes = [vp, i64, i64, vp, vp]
+            lib.i2s_oracle_act_quant.argtypes = [vp, i64, i64, vp, vp]
+            lib.i2s_oracle_gemm.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp]
+            lib.i2s_oracle_gemm_sampled.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, i64, vp, vp]
+            lib.i2s_oracle_quant_gemm.argtypes = [vp, i64, i64, vp, i64, vp, vp, vp, vp]
+            lib.i2s_oracle_ternarize_absmean.argtypes = [vp, i64, f64, vp, vp]
+            lib.i2s_oracle_dequant_f32.argtypes = [vp, i64, i64, vp]
+            for name in ("pack", "unpack", "act_quant", "gemm", "gemm_sampled", "quant_gemm",
+                         "ternarize_absmean", "dequant_f32"):
+                getattr(lib, "i2s_oracle_" + name).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise OracleError(f"oracle {what} failed with status {status}")
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def packed_bytes(n: int, k: int) -> int:
+    """Size in bytes of an I2_S tensor of n rows by k columns."""
+    return int(_load().i2s_oracle_packed_bytes(n, k))
+
+
+def pack(w: np.ndarray) -> np.ndarray:
+    """fp32 W[N,K] -> uint8 I2_S bytes (codes then the fp32 scale)."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    out = np.zeros(packed_bytes(n, k), dtype=np.uint8)
+    _check(_load().i2s_oracle_pack(_p(w), n, k, _p(out)), "pack")
+    return out
+
+
+def scale(packed: np.ndarray, n: int, k: int) -> float:
+    packed = _c(packed, np.uint8)
+    return float(_load().i2s_oracle_scale(_p(packed), n, k))
+
+
+def unpack(packed: np.ndarray, n: int, k: int) -> tuple[np.ndarray, float]:
+    """I2_S bytes -> (int8 T[N,K] in {-1,0,+1}, scale)."""
+    packed = _c(packed, np.uint8)
+    t = np.zeros((n, k), dtype=np.int8)
+    s = np.zeros(1, dtype=np.float32)
+    _check(_load().i2s_oracle_unpack(_p(packed), n, k, _p(t), _p(s)), "unpack")
+    return t, float(s[0])
+
+
+def act_quant(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 X[M,K] -> (int8 Xq[M,K], fp32 xs[M]) by per-token absmax."""
+    x = _c(x, np.float32)
+    m, k = x.shape
+    xq = np.zeros((m, k), dtype=np.int8)
+    xs = np.zeros(m, dtype=np.float32)
+    _check(_load().i2s_oracle_act_quant(_p(x), m, k, _p(xq), _p(xs)), "act_quant")
+    return xq, xs
+
+
+def gemm(packed: np.ndarray, n: int, k: int, xq: np.ndarray, xs: np.ndarray):
+    """(Y fp32 [M,N], acc int32 [M,N]) for packed W[N,K] and Xq[M,K]."""
+    packed = _c(packed, np.uint8)
+    xq = _c(xq, np.int8)
+    xs = _c(xs, np.float32)
+    m = xq.shape[0]
+    y = np.zeros((m, n), dtype=np.float32)
+    acc = np.zeros((m, n), dtype=np.int32)
+    _check(_load().i2s_oracle_gemm(_p(packed), n, k, _p(xq), _p(xs), m, _p(y), _p(acc)), "gemm")
+    return y, acc
+
+
+def gemm_sampled(packed, n, k, xq, xs, pos_m, pos_n):
+    """The outputs at positions (pos_m[i], pos_n[i]) only."""
+    packed = _c(packed, np.uint8)
+    xq = _c(xq, np.int8)
+    xs = _c(xs, np.float32)
+    pm = _c(pos_m, np.int64)
+    pn = _c(pos_n, np.int64)
+    cnt = pm.shape[0]
+    y = np.zeros(cnt, dtype=np.float32)
+    acc = np.zeros(cnt, dtype=np.int32)
+    _check(_load().i2s_oracle_gemm_sampled(_p(packed), n, k, _p(xq), _p(xs), xq.shape[0],
+                                           _p(pm), _p(pn), cnt, _p(y), _p(acc)), "gemm_sampled")
+    return y, acc
+
+
+def quant_gemm(packed, n, k, x):
+    """Per-token quantization of x then the matmul: (Y, acc, xq, xs)."""
+    packed = _c(packed, np.uint8)
+    x = _c(x, np.float32)
+    m = x.shape[0]
+    y = np.zeros((m, n), dtype=np.float32)
+    acc = np.zeros((m, n), dtype=np.int32)
+    xq = np.zeros((m, k), dtype=np.int8)
+    xs = np.zeros(m, dtype=np.float32)
+    _check(_load().i2s_oracle_quant_gemm(_p(packed), n, k, _p(x), m, _p(y), _p(acc), _p(xq),
+                                         _p(xs)), "quant_gemm")
+    return y, acc, xq, xs
+
+
+def ternarize_absmean(w: np.ndarray, eps: float = 1e-5) -> tuple[np.ndarray, float]:
+    """AbsMean RoundClip ternarization: (W~ * gamma as fp32, gamma as fp64)."""
+    w = _c(w, np.float32)
+    out = np.zeros_like(w)
+    g = np.zeros(1, dtype=np.float64)
+    _check(_load().i2s_oracle_ternarize_absmean(_p(w), w.size, float(eps), _p(out), _p(g)),
+           "ternarize_absmean")
+    return out, float(g[0])
+
+
+def dequant_f32(packed: np.ndarray, n: int, k: int) -> np.ndarray:
+    """Full-tensor I2_S -> fp32 weights (code - 1) * scale."""
+    packed = _c(packed, np.uint8)
+    out = np.zeros((n, k), dtype=np.float32)
+    _check(_load().i2s_oracle_dequant_f32(_p(packed), n, k, _p(out)), "dequant_f32")
+    return out
