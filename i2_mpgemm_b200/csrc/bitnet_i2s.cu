@@ -1,0 +1,343 @@
+// bitnet_i2s.cu -- the C ABI of include/bitnet_i2s.h: argument checks on the
+// host, tensor-map encoding, and the kernel launches.  One translation unit
+// (the kernels are header-only) so that the device error flag is a single
+// symbol.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "bitnet_i2s.h"
+#include "mma_kernel.cuh"
+#include "quant_kernels.cuh"
+
+namespace {
+
+using namespace bitnet;
+
+constexpr int64_t kMaxK = 131072;  // 127 * K < 2^24: (float)acc is exact
+constexpr int kMaxDevices = 64;
+
+thread_local std::string g_last_error;
+
+bitnet_status fail(bitnet_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+bitnet_status fail(bitnet_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+bitnet_status ok() {
+  g_last_error.clear();
+  return BITNET_OK;
+}
+
+bitnet_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BITNET_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The current device must be compute capability 10.0 (B200 class); the
+// library holds sm_100a code only.
+bitnet_status check_device(int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(BITNET_ERR_UNSUPPORTED, "device %d", dev);
+  static std::atomic<int> verdict[kMaxDevices];  // 0 unknown, 1 ok, 2 unsupported
+  int v = verdict[dev].load(std::memory_order_acquire);
+  if (v == 0) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    v = (major == 10 && minor == 0) ? 1 : 2;
+    verdict[dev].store(v, std::memory_order_release);
+  }
+  if (v != 1) return fail(BITNET_ERR_UNSUPPORTED, "device %d is not compute capability 10.0", dev);
+  *dev_out = dev;
+  return BITNET_OK;
+}
+
+// cuTensorMapEncodeTiled from the driver, without linking libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor map: `cols` bytes per row (contiguous), `rows` rows with a
+// pitch of `cols` bytes, box `box_cols` x `box_rows`, 128-byte swizzle.
+// Out-of-bounds box elements read as zero.
+bitnet_status encode_u8_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                           uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(BITNET_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BITNET_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return BITNET_OK;
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename Kernel>
+bitnet_status ensure_smem(Kernel kern, size_t bytes, int dev, std::atomic<uint8_t>* done) {
+  if (done[dev].load(std::memory_order_acquire)) return BITNET_OK;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(bytes));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  done[dev].store(1, std::memory_order_release);
+  return BITNET_OK;
+}
+
+cudaLaunchAttribute pdl_attr(bool on) {
+  cudaLaunchAttribute a;
+  std::memset(&a, 0, sizeof(a));
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = on ? 1 : 0;
+  return a;
+}
+
+template <int T, bool kCodes>
+bitnet_status launch_mma(const uint8_t* packed, int64_t n, int64_t k, const int8_t* xq,
+                         const float* xs, int64_t m, float* y, int32_t* acc, bool pdl,
+                         cudaStream_t stream, int dev) {
+  using C = MmaCfg<T, kCodes>;
+  static std::atomic<uint8_t> smem_done[kMaxDevices];
+  auto kern = i2s_mma_kernel<T, kCodes>;
+  bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
+  if (st != BITNET_OK) return st;
+  CUtensorMap tw, tx;
+  st = encode_u8_2d(&tw, packed, static_cast<uint64_t>(k / 4), static_cast<uint64_t>(n), 128, 128);
+  if (st != BITNET_OK) return st;
+  st = encode_u8_2d(&tx, xq, static_cast<uint64_t>(k), static_cast<uint64_t>(m), 128, T);
+  if (st != BITNET_OK) return st;
+  MmaParams p;
+  p.packed = packed;
+  p.xs = xs;
+  p.y = y;
+  p.acc = acc;
+  p.n = n;
+  p.k = k;
+  p.m = m;
+  p.pdl = pdl ? 1 : 0;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>((n + 127) / 128), static_cast<unsigned>((m + T - 1) / T));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr = pdl_attr(pdl);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the I2_S matmul kernel");
+  return BITNET_OK;
+}
+
+bitnet_status check_matmul_args(const char* fn, const uint8_t* packed, int64_t n, int64_t k,
+                                const void* x, const float* xs_or_dummy, int64_t m, float* y,
+                                int64_t max_m) {
+  if (packed == nullptr || x == nullptr || xs_or_dummy == nullptr || y == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+  if (n < 1 || m < 1) return fail(BITNET_ERR_SHAPE, "%s: N=%lld and M=%lld must be >= 1", fn,
+                                  (long long)n, (long long)m);
+  if (k < 128 || k % 128 != 0 || k > kMaxK)
+    return fail(BITNET_ERR_SHAPE, "%s: K=%lld must be a multiple of 128 in [128, %lld]", fn,
+                (long long)k, (long long)kMaxK);
+  if (m > max_m)
+    return fail(BITNET_ERR_SHAPE, "%s: M=%lld exceeds %lld", fn, (long long)m, (long long)max_m);
+  if (n > int64_t{0x7fffffff})
+    return fail(BITNET_ERR_SHAPE, "%s: N=%lld too large", fn, (long long)n);
+  if (!aligned(packed, 16)) return fail(BITNET_ERR_ALIGN, "%s: packed must be 16-byte aligned", fn);
+  if (!aligned(x, 16)) return fail(BITNET_ERR_ALIGN, "%s: activations must be 16-byte aligned", fn);
+  if (!aligned(y, 4) || !aligned(xs_or_dummy, 4))
+    return fail(BITNET_ERR_ALIGN, "%s: Y and xs must be 4-byte aligned", fn);
+  return BITNET_OK;
+}
+
+// Dispatch on the token count: small token tiles with the code-plus-correction
+// unpack for decode, 128-token tiles with the signed unpack for prefill.
+bitnet_status run_matmul(const uint8_t* packed, int64_t n, int64_t k, const int8_t* xq,
+                         const float* xs, int64_t m, float* y, int32_t* acc, bool pdl,
+                         cudaStream_t stream, int dev) {
+  if (m <= 16) return launch_mma<16, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
+  if (m <= 32) return launch_mma<32, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
+  if (m <= 64) return launch_mma<64, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
+  return launch_mma<128, false>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
+}
+
+constexpr int64_t kMaxTokens = int64_t{65535} * 16;  // grid.y limit at the smallest tile
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+size_t bitnet_i2s_packed_bytes(int64_t N, int64_t K) {
+  if (N < 1 || K < 128 || K % 128 != 0) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) / 4 + 4;
+}
+
+bitnet_status bitnet_i2s_pack(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                              void* stream) {
+  if (W == nullptr || packed == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_pack: null pointer argument");
+  if (N < 1 || K < 128 || K % 128 != 0 || K > kMaxK)
+    return fail(BITNET_ERR_SHAPE, "bitnet_i2s_pack: N=%lld, K=%lld (K a multiple of 128)",
+                (long long)N, (long long)K);
+  if (!aligned(W, 16) || !aligned(packed, 16))
+    return fail(BITNET_ERR_ALIGN, "bitnet_i2s_pack: W and packed must be 16-byte aligned");
+  int dev;
+  bitnet_status st = check_device(&dev);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t count = N * K;
+  uint8_t* tail = packed + count / 4;
+  cudaError_t e = cudaMemsetAsync(tail, 0, 4, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t n4 = count / 4;
+  const int grid_a = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, int64_t{sms} * 8));
+  i2s_absmax_kernel<<<grid_a, 256, 0, s>>>(reinterpret_cast<const float4*>(W), n4,
+                                           reinterpret_cast<unsigned int*>(tail));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the absmax kernel");
+  const int64_t words = count / 16;
+  const int grid_p = static_cast<int>(std::min<int64_t>((words + 255) / 256, int64_t{sms} * 16));
+  i2s_pack_kernel<<<grid_p, 256, 0, s>>>(W, words, reinterpret_cast<uint32_t*>(packed),
+                                         reinterpret_cast<const float*>(tail));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the pack kernel");
+  return ok();
+}
+
+bitnet_status bitnet_act_quant_i8(const float* X, int64_t M, int64_t K, int8_t* Xq, float* xs,
+                                  void* stream) {
+  if (X == nullptr || Xq == nullptr || xs == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_act_quant_i8: null pointer argument");
+  if (M < 1 || M > int64_t{0x7fffffff} || K < 16 || K % 16 != 0 || K > kMaxK)
+    return fail(BITNET_ERR_SHAPE, "bitnet_act_quant_i8: M=%lld, K=%lld (K a multiple of 16)",
+                (long long)M, (long long)K);
+  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(xs, 4))
+    return fail(BITNET_ERR_ALIGN, "bitnet_act_quant_i8: X and Xq must be 16-byte aligned");
+  int dev;
+  bitnet_status st = check_device(&dev);
+  if (st != BITNET_OK) return st;
+  act_quant_kernel<<<static_cast<unsigned>(M), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      X, K, Xq, xs);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the activation quant kernel");
+  return ok();
+}
+
+bitnet_status bitnet_i2s_gemv(const uint8_t* packed, int64_t N, int64_t K, const int8_t* Xq,
+                              const float* xs, int64_t M, float* Y, int32_t* acc_or_null,
+                              void* stream) {
+  bitnet_status st = check_matmul_args("bitnet_i2s_gemv", packed, N, K, Xq, xs, M, Y, 64);
+  if (st != BITNET_OK) return st;
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  st = run_matmul(packed, N, K, Xq, xs, M, Y, acc_or_null, false,
+                  static_cast<cudaStream_t>(stream), dev);
+  return st == BITNET_OK ? ok() : st;
+}
+
+bitnet_status bitnet_i2s_gemm(const uint8_t* packed, int64_t N, int64_t K, const int8_t* Xq,
+                              const float* xs, int64_t M, float* Y, int32_t* acc_or_null,
+                              void* stream) {
+  bitnet_status st = check_matmul_args("bitnet_i2s_gemm", packed, N, K, Xq, xs, M, Y, kMaxTokens);
+  if (st != BITNET_OK) return st;
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  st = run_matmul(packed, N, K, Xq, xs, M, Y, acc_or_null, false,
+                  static_cast<cudaStream_t>(stream), dev);
+  return st == BITNET_OK ? ok() : st;
+}
+
+size_t bitnet_i2s_quant_gemv_workspace_bytes(int64_t M, int64_t K) {
+  if (M < 1 || K < 128 || K % 128 != 0) return 0;
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
+         align256(static_cast<size_t>(M) * sizeof(float));
+}
+
+bitnet_status bitnet_i2s_quant_gemv(const uint8_t* packed, int64_t N, int64_t K, const float* X,
+                                    int64_t M, float* Y, int32_t* acc_or_null, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  const float* dummy_xs = reinterpret_cast<const float*>(X);
+  bitnet_status st =
+      check_matmul_args("bitnet_i2s_quant_gemv", packed, N, K, X, dummy_xs, M, Y, kMaxTokens);
+  if (st != BITNET_OK) return st;
+  if (workspace == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_quant_gemv: null workspace");
+  if (!aligned(workspace, 256))
+    return fail(BITNET_ERR_ALIGN, "bitnet_i2s_quant_gemv: workspace must be 256-byte aligned");
+  const size_t need = bitnet_i2s_quant_gemv_workspace_bytes(M, K);
+  if (workspace_bytes < need)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_quant_gemv: workspace of %zu bytes < %zu",
+                workspace_bytes, need);
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int8_t* xq = static_cast<int8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                       align256(static_cast<size_t>(M) * static_cast<size_t>(K)));
+  // Quantize with PDL: the kernel waits for whatever precedes it, then lets
+  // the matmul launch so its weight loads overlap the quantization.
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(M));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr = pdl_attr(true);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, X, K, xq, xs);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the activation quant kernel");
+  st = run_matmul(packed, N, K, xq, xs, M, Y, acc_or_null, true, s, dev);
+  return st == BITNET_OK ? ok() : st;
+}
+
+bitnet_status bitnet_device_status(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  unsigned int flags = 0;
+  e = cudaMemcpyFromSymbol(&flags, g_error_flags, sizeof(flags));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error flag");
+  if (flags != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_error_flags, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error flag");
+    return fail(BITNET_ERR_DEVICE_TIMEOUT, "a device-side wait ran out (flags 0x%x)", flags);
+  }
+  return ok();
+}
+
+const char* bitnet_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,183 @@
+"""ctypes binding of ``libbitnet_i2s.so`` (C ABI in ``include/bitnet_i2s.h``).
+
+Argument marshalling only: each function takes torch CUDA tensors, checks
+their dtype, device and layout, allocates outputs the caller did not pass,
+and calls the C entry point of the same name on the current torch stream.
+All computation happens in the library's sm_100a kernels; there is no CPU or
+PyTorch fallback.  Importing this module raises if the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LIB_PATH = _build.LIB
+
+BITNET_OK = 0
+STATUS_NAMES = {
+    0: "BITNET_OK",
+    1: "BITNET_ERR_INVALID_ARG",
+    2: "BITNET_ERR_SHAPE",
+    3: "BITNET_ERR_ALIGN",
+    4: "BITNET_ERR_CUDA",
+    5: "BITNET_ERR_DEVICE_TIMEOUT",
+    6: "BITNET_ERR_UNSUPPORTED",
+}
+
+# Every function the header declares, with its ctypes signature.
+_I64, _VP, _SZ, _I32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+SIGNATURES = {
+    "bitnet_i2s_packed_bytes": (_SZ, [_I64, _I64]),
+    "bitnet_i2s_pack": (_I32, [_VP, _I64, _I64, _VP, _VP]),
+    "bitnet_act_quant_i8": (_I32, [_VP, _I64, _I64, _VP, _VP, _VP]),
+    "bitnet_i2s_gemv": (_I32, [_VP, _I64, _I64, _VP, _VP, _I64, _VP, _VP, _VP]),
+    "bitnet_i2s_gemm": (_I32, [_VP, _I64, _I64, _VP, _VP, _I64, _VP, _VP, _VP]),
+    "bitnet_i2s_quant_gemv_workspace_bytes": (_SZ, [_I64, _I64]),
+    "bitnet_i2s_quant_gemv": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
+    "bitnet_device_status": (_I32, []),
+    "bitnet_last_error": (ctypes.c_char_p, []),
+}
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"CUDA library {path} is missing; build it with `python -m i2_mpgemm_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = load_library()
+
+
+def _check(status: int) -> None:
+    if status != BITNET_OK:
+        raise BitnetError(status, lib.bitnet_last_error().decode(errors="replace"))
+
+
+def _stream(stream) -> int | None:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream or None
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, numel: int | None = None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs {numel}")
+
+
+def bitnet_i2s_packed_bytes(n: int, k: int) -> int:
+    return int(lib.bitnet_i2s_packed_bytes(n, k))
+
+
+def bitnet_i2s_pack(w: torch.Tensor, packed: torch.Tensor | None = None, stream=None):
+    """fp32 W[N,K] -> uint8 I2_S tensor of bitnet_i2s_packed_bytes(N,K) bytes."""
+    _need(w, "W", torch.float32)
+    n, k = w.shape
+    nbytes = bitnet_i2s_packed_bytes(n, k)
+    if packed is None:
+        packed = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=w.device)
+    _need(packed, "packed", torch.uint8, nbytes)
+    _check(lib.bitnet_i2s_pack(_ptr(w), n, k, _ptr(packed), _stream(stream)))
+    return packed
+
+
+def bitnet_act_quant_i8(x: torch.Tensor, xq: torch.Tensor | None = None,
+                        xs: torch.Tensor | None = None, stream=None):
+    """fp32 X[M,K] -> (int8 Xq[M,K], fp32 xs[M])."""
+    _need(x, "X", torch.float32)
+    m, k = x.shape
+    xq = torch.empty((m, k), dtype=torch.int8, device=x.device) if xq is None else xq
+    xs = torch.empty(m, dtype=torch.float32, device=x.device) if xs is None else xs
+    _need(xq, "Xq", torch.int8, m * k)
+    _need(xs, "xs", torch.float32, m)
+    _check(lib.bitnet_act_quant_i8(_ptr(x), m, k, _ptr(xq), _ptr(xs), _stream(stream)))
+    return xq, xs
+
+
+def _matmul(fn, packed, n, k, xq, xs, y, acc, want_acc, stream):
+    _need(packed, "packed", torch.uint8, bitnet_i2s_packed_bytes(n, k))
+    _need(xq, "Xq", torch.int8)
+    m = xq.shape[0]
+    _need(xq, "Xq", torch.int8, m * k)
+    _need(xs, "xs", torch.float32, m)
+    dev = packed.device
+    y = torch.empty((m, n), dtype=torch.float32, device=dev) if y is None else y
+    _need(y, "Y", torch.float32, m * n)
+    if want_acc and acc is None:
+        acc = torch.empty((m, n), dtype=torch.int32, device=dev)
+    if acc is not None:
+        _need(acc, "acc", torch.int32, m * n)
+    _check(fn(_ptr(packed), n, k, _ptr(xq), _ptr(xs), m, _ptr(y), _ptr(acc), _stream(stream)))
+    return (y, acc) if acc is not None else y
+
+
+def bitnet_i2s_gemv(packed, n, k, xq, xs, y=None, acc=None, want_acc=False, stream=None):
+    """Decode matmul (M = Xq.shape[0] in 1..64): Y, or (Y, acc) with want_acc."""
+    return _matmul(lib.bitnet_i2s_gemv, packed, n, k, xq, xs, y, acc, want_acc, stream)
+
+
+def bitnet_i2s_gemm(packed, n, k, xq, xs, y=None, acc=None, want_acc=False, stream=None):
+    """Matmul for any M >= 1: Y, or (Y, acc) with want_acc."""
+    return _matmul(lib.bitnet_i2s_gemm, packed, n, k, xq, xs, y, acc, want_acc, stream)
+
+
+def bitnet_i2s_quant_gemv_workspace_bytes(m: int, k: int) -> int:
+    return int(lib.bitnet_i2s_quant_gemv_workspace_bytes(m, k))
+
+
+def bitnet_i2s_quant_gemv(packed, n, k, x, y=None, acc=None, workspace=None, want_acc=False,
+                          stream=None):
+    """Per-token quantization of fp32 X[M,K] then the matmul: Y or (Y, acc)."""
+    _need(packed, "packed", torch.uint8, bitnet_i2s_packed_bytes(n, k))
+    _need(x, "X", torch.float32)
+    m = x.shape[0]
+    _need(x, "X", torch.float32, m * k)
+    dev = packed.device
+    wsb = bitnet_i2s_quant_gemv_workspace_bytes(m, k)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8)
+    y = torch.empty((m, n), dtype=torch.float32, device=dev) if y is None else y
+    _need(y, "Y", torch.float32, m * n)
+    if want_acc and acc is None:
+        acc = torch.empty((m, n), dtype=torch.int32, device=dev)
+    if acc is not None:
+        _need(acc, "acc", torch.int32, m * n)
+    _check(lib.bitnet_i2s_quant_gemv(_ptr(packed), n, k, _ptr(x), m, _ptr(y), _ptr(acc),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)))
+    return (y, acc) if acc is not None else y
+
+
+def bitnet_device_status() -> None:
+    """Synchronize and raise BitnetError if a device-side wait ran out."""
+    _check(lib.bitnet_device_status())
+
+
+def bitnet_last_error() -> str:
+    return lib.bitnet_last_error().decode(errors="replace")

@@ -1,0 +1,149 @@
+/*
+ * bitnet_i2s.h -- C ABI of the B200 (sm_100a) I2_S ternary x int8 matmul.
+ *
+ * The library computes, for ternary weights w[n,k] in {-1,0,+1} packed two
+ * bits each with one fp32 per-tensor scale s, and per-token int8 activations
+ * xq[m,k] with fp32 scales xs[m]:
+ *
+ *     acc[m,n] = sum_k w[n,k] * xq[m,k]            (exact int32)
+ *     y[m,n]   = ((float)acc[m,n] * xs[m]) * s     (two fp32 multiplies)
+ *
+ * Sources (web pages, cited by title and section):
+ *   [P1] "How BitNet's 1-Bit (I2_S) Quantization Works Compared to Standard
+ *        LLM Quantization": sections "Ternary Representation and Packing",
+ *        "Per-Tensor Scaling Strategy", "How I2_S Kernels Process the Format".
+ *   [P2] "BitNet Inference Preprocessing: Converting Hugging Face Checkpoints
+ *        to I2S GGUF": "The Two-Stage BitNet Inference Preprocessing
+ *        Pipeline" (the packing is lossless; the seven ternary projections).
+ *   [P3] "ik_llama.cpp 运行 BitNet b1.58 2B 模型实战：从 bitnet-b1.58 架构兼容到
+ *        I2_S 量化转换": section 5.1 (I2_S tensors are dequantized to f32 in
+ *        full before requantizing).
+ *   [P5] "LLM Quantization Paradigms: FP8, AWQ, EXL2 & BitNet b1.58 in 2026":
+ *        section 5, figure "BitNet b1.58 Ternary Matrix Multiplication" and
+ *        "The Mathematics of BitNet b1.58".
+ *
+ * I2_S byte layout (the packed tensor of an N x K weight matrix, K % 128 == 0):
+ *   bytes [0, N*K/4): 2-bit codes, code = w + 1 (so -1,0,+1 -> 0,1,2; code 3
+ *     never occurs).  Weights are taken in row-major order in blocks of 128;
+ *     weight j of a block sits in byte j % 32 of the block's 32 bytes, in
+ *     bits [7-2g : 6-2g] with g = j / 32 (the shift 6 - 2*group of [P1]).
+ *   bytes [N*K/4, N*K/4 + 4): the scale s = max|W| as little-endian fp32 [P1].
+ *
+ * Conventions for every call below:
+ *   - Pointers are DEVICE pointers, allocated and owned by the caller; the
+ *     library never allocates, frees or keeps them.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on that stream; arguments are
+ *     checked on the host before anything is launched.
+ *   - The current CUDA device must be a B200-class GPU (sm_100a); the
+ *     pointers must belong to it.
+ *   - Return value: BITNET_OK, or an error code with a message readable from
+ *     bitnet_last_error() (thread-local; valid until the next call on the
+ *     same thread).  On an argument error nothing is launched.
+ *   - Device-side waits are bounded.  A wait that runs out (about two
+ *     seconds) makes the kernel stop early and raise a device error flag;
+ *     bitnet_device_status() reports and clears it.
+ *   - Shape limits: 1 <= N, M; K a multiple of 128 with K <= 131072, which
+ *     keeps |acc| <= 127*K < 2^24 so (float)acc is exact.
+ */
+#ifndef BITNET_I2S_H
+#define BITNET_I2S_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BITNET_API __attribute__((visibility("default")))
+#else
+#define BITNET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bitnet_status {
+  BITNET_OK = 0,
+  BITNET_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad buffer size */
+  BITNET_ERR_SHAPE = 2,         /* N, M < 1; K not a multiple of 128; over a limit */
+  BITNET_ERR_ALIGN = 3,         /* a pointer misses its required alignment */
+  BITNET_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  BITNET_ERR_DEVICE_TIMEOUT = 5,/* a bounded device-side wait ran out */
+  BITNET_ERR_UNSUPPORTED = 6    /* the current device is not sm_100 */
+} bitnet_status;
+
+/* Size in bytes of the I2_S tensor of an N x K weight matrix: N*K/4 code
+ * bytes plus the 4-byte scale [P1 "Ternary Representation and Packing",
+ * "Per-Tensor Scaling Strategy"].  Returns 0 for an invalid shape. */
+BITNET_API size_t bitnet_i2s_packed_bytes(int64_t N, int64_t K);
+
+/* Pack fp32 weights W[N,K] (row-major) into I2_S [P1 "Ternary Representation
+ * and Packing", "Per-Tensor Scaling Strategy"; P2: lossless for weights that
+ * are already ternary times one scale].
+ *   s = max|W|; each weight becomes q = clip(round_half_away(W/s), -1, 1)
+ *   (fp32 IEEE divide; s == 0 gives q = 0 everywhere) and code q + 1.
+ * W: N*K fp32, 16-byte aligned.  packed: bitnet_i2s_packed_bytes(N,K)
+ * bytes, 16-byte aligned; fully overwritten (codes and scale). */
+BITNET_API bitnet_status bitnet_i2s_pack(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                              void* stream);
+
+/* Per-token absmax int8 quantization [P5 section 5, "The Mathematics of
+ * BitNet b1.58"]: for each row m of X[M,K] (row-major fp32),
+ *   amax = max_k |x|; xq = clamp(round_half_even(x * (127/amax)), -127, 127);
+ *   xs[m] = amax / 127 (fp32 IEEE divides); a zero row gives xq = 0, xs = 0.
+ * X: 16-byte aligned; K % 16 == 0.  Xq: M*K int8, 16-byte aligned.
+ * xs: M fp32. */
+BITNET_API bitnet_status bitnet_act_quant_i8(const float* X, int64_t M, int64_t K, int8_t* Xq, float* xs,
+                                  void* stream);
+
+/* Decode-shaped ternary matmul, M = 1..64 tokens [P5 section 5 figure, "BitNet
+ * b1.58 Ternary Matrix Multiplication" (add, subtract or skip per ternary
+ * weight, integer accumulation); P1 "How I2_S Kernels Process the Format"
+ * (unpack the 2-bit codes, multiply by the shared per-tensor scale)].
+ *   packed: I2_S tensor of W[N,K] (as written by bitnet_i2s_pack), 16-byte
+ *           aligned; the scale is read from its tail.
+ *   Xq:     M*K int8 row-major, 16-byte aligned.   xs: M fp32.
+ *   Y:      M*N fp32 row-major (token-major), written.
+ *   acc_or_null: if not NULL, M*N int32 row-major receives the exact
+ *           accumulators.
+ * Memory-bound: streams N*K/4 packed bytes once. */
+BITNET_API bitnet_status bitnet_i2s_gemv(const uint8_t* packed, int64_t N, int64_t K, const int8_t* Xq,
+                              const float* xs, int64_t M, float* Y, int32_t* acc_or_null,
+                              void* stream);
+
+/* The same contraction for any M >= 1 (prefill), with the same arguments and
+ * results; for M > 64 it uses a tile shaped for tensor-core throughput. */
+BITNET_API bitnet_status bitnet_i2s_gemm(const uint8_t* packed, int64_t N, int64_t K, const int8_t* Xq,
+                              const float* xs, int64_t M, float* Y, int32_t* acc_or_null,
+                              void* stream);
+
+/* Bytes of device scratch that bitnet_i2s_quant_gemv needs for M tokens of
+ * length K (the int8 activations and their scales).  0 for a bad shape. */
+BITNET_API size_t bitnet_i2s_quant_gemv_workspace_bytes(int64_t M, int64_t K);
+
+/* Activation quantization followed by the ternary matmul: exactly
+ * bitnet_act_quant_i8(X) then bitnet_i2s_gemm [P5 section 5: activations
+ * quantized per token with AbsMax, then the ternary contraction].
+ *   X: M*K fp32 row-major, 16-byte aligned.
+ *   workspace: caller-owned device scratch of at least
+ *     bitnet_i2s_quant_gemv_workspace_bytes(M,K) bytes, 256-byte aligned;
+ *     it must not be used by other work that may run at the same time.
+ *   Other arguments as bitnet_i2s_gemv; M >= 1. */
+BITNET_API bitnet_status bitnet_i2s_quant_gemv(const uint8_t* packed, int64_t N, int64_t K, const float* X,
+                                    int64_t M, float* Y, int32_t* acc_or_null, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* Waits for all work on the current device, then returns
+ * BITNET_ERR_DEVICE_TIMEOUT if any kernel of this library gave up on a
+ * bounded wait since the last call (and clears the flag), BITNET_ERR_CUDA if
+ * the device reports an error, else BITNET_OK. */
+BITNET_API bitnet_status bitnet_device_status(void);
+
+/* Message of the last error on this thread ("" if none). */
+BITNET_API const char* bitnet_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_I2S_H */

@@ -1,0 +1,110 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before touching CUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names.update(re.findall(r"BITNET_API\s+[\w\s\*]+?\b(bitnet_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def i2s():
+    from i2_mpgemm_b200 import build
+    build.build()
+    from i2_mpgemm_b200 import i2s as mod
+    return mod
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("bitnet_i2s_packed_bytes", "bitnet_i2s_pack", "bitnet_act_quant_i8",
+                     "bitnet_i2s_gemv", "bitnet_i2s_gemm", "bitnet_i2s_quant_gemv",
+                     "bitnet_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(i2s):
+    lib = ctypes.CDLL(i2s.LIB_PATH)
+    names = declared_functions()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    # the binding wraps exactly the declared functions
+    assert set(i2s.SIGNATURES) == names
+
+
+def test_size_helpers(i2s):
+    assert i2s.bitnet_i2s_packed_bytes(640, 2560) == 640 * 2560 // 4 + 4
+    assert i2s.bitnet_i2s_packed_bytes(1, 100) == 0
+    assert i2s.bitnet_i2s_packed_bytes(0, 128) == 0
+    ws = i2s.bitnet_i2s_quant_gemv_workspace_bytes(3, 256)
+    assert ws >= 3 * 256 + 3 * 4 and ws % 256 == 0
+    assert i2s.bitnet_i2s_quant_gemv_workspace_bytes(0, 256) == 0
+
+
+def _call(i2s, name, *args):
+    return getattr(i2s.lib, name)(*args)
+
+
+A = 1 << 20  # a 256-byte aligned fake address: never dereferenced, checks fail first
+
+
+def test_matmul_argument_errors_on_host(i2s):
+    for fn in ("bitnet_i2s_gemv", "bitnet_i2s_gemm"):
+        # null pointers
+        assert _call(i2s, fn, None, 8, 128, A, A, 1, A, None, None) == 1
+        assert _call(i2s, fn, A, 8, 128, None, A, 1, A, None, None) == 1
+        assert _call(i2s, fn, A, 8, 128, A, None, 1, A, None, None) == 1
+        assert _call(i2s, fn, A, 8, 128, A, A, 1, None, None, None) == 1
+        # shapes
+        assert _call(i2s, fn, A, 0, 128, A, A, 1, A, None, None) == 2
+        assert _call(i2s, fn, A, 8, 128, A, A, 0, A, None, None) == 2
+        assert _call(i2s, fn, A, 8, 100, A, A, 1, A, None, None) == 2
+        assert _call(i2s, fn, A, 8, 0, A, A, 1, A, None, None) == 2
+        assert _call(i2s, fn, A, 8, 262144, A, A, 1, A, None, None) == 2
+        # alignment
+        assert _call(i2s, fn, A + 8, 8, 128, A, A, 1, A, None, None) == 3
+        assert _call(i2s, fn, A, 8, 128, A + 4, A, 1, A, None, None) == 3
+        assert _call(i2s, fn, A, 8, 128, A, A, 1, A + 2, None, None) == 3
+        assert "aligned" in i2s.bitnet_last_error()
+    # decode entry is limited to 64 tokens
+    assert _call(i2s, "bitnet_i2s_gemv", A, 8, 128, A, A, 65, A, None, None) == 2
+
+
+def test_pack_and_quant_argument_errors_on_host(i2s):
+    assert _call(i2s, "bitnet_i2s_pack", None, 4, 128, A, None) == 1
+    assert _call(i2s, "bitnet_i2s_pack", A, 4, 96, A, None) == 2
+    assert _call(i2s, "bitnet_i2s_pack", A + 4, 4, 128, A, None) == 3
+    assert _call(i2s, "bitnet_act_quant_i8", A, 2, 24, A, A, None) == 2
+    assert _call(i2s, "bitnet_act_quant_i8", A, 0, 32, A, A, None) == 2
+    assert _call(i2s, "bitnet_act_quant_i8", A + 4, 2, 32, A, A, None) == 3
+    assert _call(i2s, "bitnet_act_quant_i8", A, 2, 32, None, A, None) == 1
+    fn = "bitnet_i2s_quant_gemv"
+    need = i2s.bitnet_i2s_quant_gemv_workspace_bytes(2, 128)
+    assert _call(i2s, fn, A, 8, 128, A, 2, A, None, None, need, None) == 1
+    assert _call(i2s, fn, A, 8, 128, A, 2, A, None, A + 16, need, None) == 3
+    assert _call(i2s, fn, A, 8, 128, A, 2, A, None, A, need - 1, None) == 1
+    assert "workspace" in i2s.bitnet_last_error()
+
+
+def test_product_package_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "i2_mpgemm_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
+                assert "i2s_oracle" not in text, f

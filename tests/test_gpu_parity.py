@@ -1,0 +1,274 @@
+"""GPU parity: every C entry point against the CPU oracle on the same seeded inputs.
+
+int32 accumulators and int8/byte outputs must be bit-exact; fp32 outputs
+within 1e-5 relative error (tests/parity.py).  Small shapes are compared in
+full and span several 128-row tiles, several token tiles and ragged tails in
+N, M and K; the workload sizes are compared on sampled outputs (computed one
+by one by the oracle) plus an exact whole-output identity.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from i2_mpgemm_b200 import inputs
+from tests.parity import assert_acc_equal, assert_y_close, column_sum_identity, sample_positions
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def i2s():
+    from i2_mpgemm_b200 import i2s as mod
+    return mod
+
+
+def dev(t):
+    return t.contiguous().cuda()
+
+
+# ------------------------------------------------------------------- pack
+
+PACK_SHAPES = [(1, 128), (7, 384), (130, 640), (300, 1152), (640, 2560), (33, 6912)]
+
+
+@pytest.mark.parametrize("n,k", PACK_SHAPES)
+def test_pack_is_byte_exact_on_ternary_weights(i2s, n, k):
+    w, _, _ = inputs.ternary_weights(n, k, 5000 + n + k)
+    got = i2s.bitnet_i2s_pack(dev(w)).cpu().numpy()
+    assert np.array_equal(got, oracle.pack(w.numpy()))
+
+
+@pytest.mark.parametrize("n,k", PACK_SHAPES[:4])
+def test_pack_is_byte_exact_on_arbitrary_weights(i2s, n, k):
+    w = torch.randn((n, k), generator=torch.Generator().manual_seed(n * k))
+    w[0, 0] = 3.0  # a known maximum; values near +-1.5 exercise the rounding
+    w[:, 1] = 1.5
+    got = i2s.bitnet_i2s_pack(dev(w)).cpu().numpy()
+    assert np.array_equal(got, oracle.pack(w.numpy()))
+
+
+def test_pack_of_zero_tensor(i2s):
+    got = i2s.bitnet_i2s_pack(torch.zeros((3, 256), device="cuda")).cpu().numpy()
+    assert np.array_equal(got, oracle.pack(np.zeros((3, 256), np.float32)))
+
+
+def test_pack_of_every_projection_shape(i2s):
+    for idx, p in enumerate(inputs.projections_2b()):
+        w, _, _ = inputs.ternary_weights(p.n, p.k, inputs.seed_layer(idx))
+        got = i2s.bitnet_i2s_pack(dev(w)).cpu().numpy()
+        assert np.array_equal(got, oracle.pack(w.numpy())), p.name
+
+
+# -------------------------------------------------------- activation quant
+
+@pytest.mark.parametrize("m,k,outliers", [(1, 2560, False), (4, 6912, False), (16, 2560, True),
+                                          (37, 384, False), (3, 16, False), (2, 28672, True)])
+def test_act_quant_is_bit_exact(i2s, m, k, outliers):
+    x = inputs.activations(m, k, 700 + m + k, outliers=outliers)
+    xq, xs = i2s.bitnet_act_quant_i8(dev(x))
+    xq_ref, xs_ref = oracle.act_quant(x.numpy())
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(xs.cpu().numpy(), xs_ref)
+
+
+def test_act_quant_worked_examples_and_zero_rows(i2s):
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "act_quant_worked_examples.json")
+    for ex in json.load(open(path))["examples"]:
+        x = np.zeros((1, 16), np.float32)
+        row = np.array(ex["x"][0], np.float32)
+        x[0, :row.size] = row  # zero padding leaves amax unchanged
+        xq, xs = i2s.bitnet_act_quant_i8(dev(torch.from_numpy(x)))
+        assert xq.cpu().numpy()[0, :row.size].tolist() == ex["xq"][0]
+        assert xs.cpu().numpy().tolist() == ex["xs"]
+
+
+# ------------------------------------------------------------- matmul, full
+
+# (M, N, K): several 128-row tiles with ragged N, every token tile size with
+# ragged M, and K with a partial last 512-wide stage.
+SMALL = [(1, 1, 128), (1, 7, 640), (3, 130, 384), (16, 300, 1152), (17, 129, 640),
+         (33, 257, 512), (64, 200, 1024), (65, 131, 640), (130, 300, 896), (200, 64, 256)]
+
+
+def _case(m, n, k, seed):
+    w, t, s = inputs.ternary_weights(n, k, seed)
+    x = inputs.activations(m, k, seed, outliers=(seed % 2 == 0))
+    packed = oracle.pack(w.numpy())
+    xq, xs = oracle.act_quant(x.numpy())
+    return w, t, x, packed, xq, xs
+
+
+@pytest.mark.parametrize("m,n,k", SMALL)
+def test_matmul_entries_match_oracle_in_full(i2s, m, n, k):
+    w, t, x, packed, xq, xs = _case(m, n, k, 31 * m + n + k)
+    y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+    d_packed = dev(torch.from_numpy(packed))
+    d_xq, d_xs = dev(torch.from_numpy(xq)), dev(torch.from_numpy(xs))
+    entries = [("gemm", i2s.bitnet_i2s_gemm)] + ([("gemv", i2s.bitnet_i2s_gemv)] if m <= 64 else [])
+    for name, fn in entries:
+        y, acc = fn(d_packed, n, k, d_xq, d_xs, want_acc=True)
+        assert_acc_equal(acc.cpu().numpy(), acc_ref, name)
+        assert_y_close(y.cpu().numpy(), y_ref, name)
+    y, acc = i2s.bitnet_i2s_quant_gemv(d_packed, n, k, dev(x), want_acc=True)
+    assert_acc_equal(acc.cpu().numpy(), acc_ref, "quant_gemv")
+    assert_y_close(y.cpu().numpy(), y_ref, "quant_gemv")
+
+
+def test_y_without_acc_and_repeat_calls_agree(i2s):
+    m, n, k = 5, 300, 640
+    _, _, x, packed, xq, xs = _case(m, n, k, 9)
+    d_packed = dev(torch.from_numpy(packed))
+    y1 = i2s.bitnet_i2s_quant_gemv(d_packed, n, k, dev(x))
+    y2 = i2s.bitnet_i2s_quant_gemv(d_packed, n, k, dev(x))
+    assert torch.equal(y1, y2)
+    y_ref, _ = oracle.gemm(packed, n, k, xq, xs)
+    assert_y_close(y1.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("sign", [1, -1, 0])
+@pytest.mark.parametrize("m", [1, 20, 130])
+def test_closed_forms_on_gpu(i2s, sign, m):
+    n, k = 140, 768
+    w = torch.full((n, k), float(sign))
+    xq = torch.randint(-127, 128, (m, k), generator=torch.Generator().manual_seed(m),
+                       dtype=torch.int8)
+    xs = torch.ones(m)
+    _, acc = i2s.bitnet_i2s_gemm(i2s.bitnet_i2s_pack(dev(w)), n, k, dev(xq), dev(xs),
+                                 want_acc=True)
+    want = sign * xq.to(torch.int64).sum(dim=1)
+    assert torch.equal(acc.cpu().to(torch.int64), want[:, None].expand(m, n))
+
+
+def test_identity_weights_on_gpu(i2s):
+    k = 256
+    xq = torch.randint(-127, 128, (70, k), generator=torch.Generator().manual_seed(2),
+                       dtype=torch.int8)
+    _, acc = i2s.bitnet_i2s_gemm(i2s.bitnet_i2s_pack(dev(torch.eye(k))), k, k, dev(xq),
+                                 dev(torch.ones(70)), want_acc=True)
+    assert torch.equal(acc.cpu(), xq.to(torch.int32))
+
+
+def test_int32_range_at_longest_reduction_on_gpu(i2s):
+    k = 28672
+    w = torch.ones((3, k))
+    w[1] = -1.0
+    xq = torch.full((2, k), 127, dtype=torch.int8)
+    xq[1] = -127
+    _, acc = i2s.bitnet_i2s_gemv(i2s.bitnet_i2s_pack(dev(w)), 3, k, dev(xq), dev(torch.ones(2)),
+                                 want_acc=True)
+    assert acc.cpu().tolist() == [[3641344, -3641344, 3641344], [-3641344, 3641344, -3641344]]
+
+
+def test_largest_k(i2s):
+    m, n, k = 2, 130, 131072
+    _, _, x, packed, xq, xs = _case(m, n, k, 77)
+    y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+    y, acc = i2s.bitnet_i2s_quant_gemv(dev(torch.from_numpy(packed)), n, k, dev(x), want_acc=True)
+    assert_acc_equal(acc.cpu().numpy(), acc_ref)
+    assert_y_close(y.cpu().numpy(), y_ref)
+
+
+# ---------------------------------------------------- the named workloads
+
+def _packed_pair(i2s, w):
+    """(oracle bytes, device bytes) of one weight tensor; the GPU pack must be
+    byte-exact.  Oracle inputs always come from the oracle's own pack."""
+    packed = oracle.pack(w.numpy())
+    d_packed = i2s.bitnet_i2s_pack(dev(w))
+    assert np.array_equal(d_packed.cpu().numpy(), packed)
+    return packed, d_packed
+
+
+def _check_full(i2s, packed, d_packed, n, k, x, what):
+    y_ref, acc_ref, _, _ = oracle.quant_gemm(packed, n, k, x.numpy())
+    y, acc = i2s.bitnet_i2s_quant_gemv(d_packed, n, k, dev(x), want_acc=True)
+    assert_acc_equal(acc.cpu().numpy(), acc_ref, what)
+    assert_y_close(y.cpu().numpy(), y_ref, what)
+    return y, acc
+
+
+def _check_sampled(i2s, packed, d_packed, n, k, x, t, count, seed, what):
+    """quant_gemv at full size: sampled outputs against the oracle, plus the
+    exact column-sum identity over every output."""
+    m = x.shape[0]
+    y, acc = i2s.bitnet_i2s_quant_gemv(d_packed, n, k, dev(x), want_acc=True)
+    xq, xs = oracle.act_quant(x.numpy())
+    pm, pn = sample_positions(m, n, count, seed)
+    y_ref, acc_ref = oracle.gemm_sampled(packed, n, k, xq, xs, pm, pn)
+    acc_h, y_h = acc.cpu(), y.cpu()
+    assert_acc_equal(acc_h.numpy()[pm, pn], acc_ref, what)
+    assert_y_close(y_h.numpy()[pm, pn], y_ref, what)
+    assert column_sum_identity(acc_h, torch.from_numpy(xq), t), what
+
+
+def test_single_k_proj_gemv_in_full(i2s):
+    n, k = 640, 2560
+    w, t, s = inputs.ternary_weights(n, k, inputs.seed_single())
+    x = inputs.activations(1, k, inputs.seed_single())
+    packed, d_packed = _packed_pair(i2s, w)
+    y, acc = _check_full(i2s, packed, d_packed, n, k, x, "k_proj")
+    xq, xs = oracle.act_quant(x.numpy())
+    y2, acc2 = i2s.bitnet_i2s_gemv(d_packed, n, k, dev(torch.from_numpy(xq)),
+                                   dev(torch.from_numpy(xs)), want_acc=True)
+    assert torch.equal(acc2.cpu(), acc.cpu()) and torch.equal(y2.cpu(), y.cpu())
+
+
+def test_one_layer_decode_with_outliers_in_full(i2s):
+    for idx, p in enumerate(inputs.projections_2b()):
+        seed = inputs.seed_layer(idx)
+        w, t, s = inputs.ternary_weights(p.n, p.k, seed)
+        x = inputs.activations(1, p.k, seed, outliers=True)
+        packed, d_packed = _packed_pair(i2s, w)
+        _check_full(i2s, packed, d_packed, p.n, p.k, x, p.name)
+
+
+@pytest.mark.parametrize("m", [1, 4, 16])
+def test_stack_first_layer_in_full(i2s, m):
+    for idx, p in enumerate(inputs.projections_2b()):
+        seed = inputs.seed_stack(0, idx)
+        w, t, s = inputs.ternary_weights(p.n, p.k, seed)
+        x = inputs.activations(m, p.k, seed)
+        packed, d_packed = _packed_pair(i2s, w)
+        _check_full(i2s, packed, d_packed, p.n, p.k, x, f"{p.name} M={m}")
+
+
+def test_stack_all_layers_sampled(i2s):
+    for layer in range(inputs.LAYERS_2B):
+        for idx, p in enumerate(inputs.projections_2b()):
+            seed = inputs.seed_stack(layer, idx)
+            w, t, s = inputs.ternary_weights(p.n, p.k, seed)
+            packed, d_packed = _packed_pair(i2s, w)
+            for m in (1, 16):
+                x = inputs.activations(m, p.k, seed)
+                _check_sampled(i2s, packed, d_packed, p.n, p.k, x, t, 64, seed + m,
+                               f"layer {layer} {p.name} M={m}")
+
+
+@pytest.mark.parametrize("m", [512, 2048])
+def test_prefill_shapes_sampled(i2s, m):
+    shapes = [("gate", 6912, 2560), ("up", 6912, 2560), ("down", 2560, 6912)]
+    for idx, (name, n, k) in enumerate(shapes):
+        seed = inputs.seed_prefill(idx)
+        w, t, s = inputs.ternary_weights(n, k, seed)
+        x = inputs.activations(m, k, seed)
+        packed, d_packed = _packed_pair(i2s, w)
+        _check_sampled(i2s, packed, d_packed, n, k, x, t, 2048, seed, f"{name} M={m}")
+
+
+@pytest.mark.parametrize("m", [1, 64])
+def test_large_layer_sampled(i2s, m):
+    for idx, p in enumerate(inputs.projections_large()):
+        seed = inputs.seed_large(idx)
+        w, t, s = inputs.ternary_weights(p.n, p.k, seed)
+        x = inputs.activations(m, p.k, seed)
+        packed, d_packed = _packed_pair(i2s, w)
+        _check_sampled(i2s, packed, d_packed, p.n, p.k, x, t, 1024, seed + m, f"{p.name} M={m}")
+        del d_packed
+    torch.cuda.empty_cache()
+
+
+def test_no_device_wait_timed_out(i2s):
+    i2s.bitnet_device_status()
