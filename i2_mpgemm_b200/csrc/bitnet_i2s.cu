@@ -13,6 +13,7 @@
 #include <string>
 
 #include "bitnet_i2s.h"
+#include "gemv_kernel.cuh"
 #include "mma_kernel.cuh"
 #include "quant_kernels.cuh"
 
@@ -179,11 +180,110 @@ bitnet_status check_matmul_args(const char* fn, const uint8_t* packed, int64_t n
   return BITNET_OK;
 }
 
+int sm_count(int dev) {
+  static std::atomic<int> cached[kMaxDevices];
+  int v = cached[dev].load(std::memory_order_acquire);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cached[dev].store(v, std::memory_order_release);
+  }
+  return v;
+}
+
+// The integer-ALU kernel serves one or two tokens with K up to 8192 (the
+// activations of one problem live in registers); everything else goes to the
+// tensor-core kernel.
+constexpr int64_t kDp4aMaxK = 8192;
+bool use_dp4a(int64_t m, int64_t kmax) { return m >= 1 && m <= 2 && kmax <= kDp4aMaxK; }
+
+// Split every problem into work items of consecutive rows: about one item
+// per SM over the whole batch, never more than one 32 KB stage per item.
+template <int CAP>
+bitnet_status plan_items(BatchParamsT<CAP>& bp, int sms) {
+  int64_t total_rows = 0;
+  for (int i = 0; i < bp.count; ++i) total_rows += bp.p[i].n;
+  const int64_t target = std::max<int64_t>(1, (total_rows + sms - 1) / sms);
+  int64_t items = 0;
+  for (int i = 0; i < bp.count; ++i) {
+    BatchProblem& q = bp.p[i];
+    const int64_t cap = std::max<int64_t>(1, 32768 / (q.k / 4));
+    const int64_t rpi = std::min(target, cap);
+    q.rows_per_item = static_cast<int32_t>(rpi);
+    q.item_start = static_cast<int32_t>(items);
+    items += (q.n + rpi - 1) / rpi;
+    if (items > int64_t{0x7fffffff}) return fail(BITNET_ERR_SHAPE, "too many rows in one batch");
+  }
+  bp.total_items = static_cast<int32_t>(items);
+  return BITNET_OK;
+}
+
+template <int MT, int WPL, int CAP>
+bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, int grid, cudaStream_t stream, bool pdl,
+                            int dev) {
+  using C = GemvCfg<MT, WPL>;
+  static std::atomic<uint8_t> smem_done[kMaxDevices];
+  auto kern = i2s_gemv_dp4a_kernel<MT, WPL, CAP>;
+  bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
+  if (st != BITNET_OK) return st;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr = pdl_attr(pdl);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, bp);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the I2_S decode kernel");
+  return BITNET_OK;
+}
+
+template <int CAP>
+bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev) {
+  const int sms = sm_count(dev);
+  bitnet_status st = plan_items(bp, sms);
+  if (st != BITNET_OK) return st;
+  int kmax = 0;
+  for (int i = 0; i < bp.count; ++i) kmax = std::max(kmax, bp.p[i].k);
+  bp.pdl = pdl ? 1 : 0;
+  const int grid = std::min(bp.total_items, sms);
+  if (bp.m == 1)
+    return kmax <= 4096 ? launch_dp4a_t<1, 8, CAP>(bp, grid, stream, pdl, dev)
+                        : launch_dp4a_t<1, 16, CAP>(bp, grid, stream, pdl, dev);
+  return kmax <= 4096 ? launch_dp4a_t<2, 8, CAP>(bp, grid, stream, pdl, dev)
+                      : launch_dp4a_t<2, 16, CAP>(bp, grid, stream, pdl, dev);
+}
+
+BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const float* x,
+                          const int8_t* xq, const float* xs, float* y, int32_t* acc) {
+  BatchProblem q;
+  q.packed = packed;
+  q.x = x;
+  q.xq = const_cast<int8_t*>(xq);
+  q.xs = const_cast<float*>(xs);
+  q.y = y;
+  q.acc = acc;
+  q.n = static_cast<int32_t>(n);
+  q.k = static_cast<int32_t>(k);
+  q.rows_per_item = 0;
+  q.item_start = 0;
+  return q;
+}
+
 // Dispatch on the token count: small token tiles with the code-plus-correction
 // unpack for decode, 128-token tiles with the signed unpack for prefill.
 bitnet_status run_matmul(const uint8_t* packed, int64_t n, int64_t k, const int8_t* xq,
                          const float* xs, int64_t m, float* y, int32_t* acc, bool pdl,
                          cudaStream_t stream, int dev) {
+  if (use_dp4a(m, k)) {
+    BatchParamsT<1> bp;
+    bp.count = 1;
+    bp.m = static_cast<int32_t>(m);
+    bp.p[0] = make_problem(packed, n, k, nullptr, xq, xs, y, acc);
+    return launch_dp4a(bp, stream, pdl, dev);
+  }
   if (m <= 16) return launch_mma<16, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
   if (m <= 32) return launch_mma<32, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
   if (m <= 64) return launch_mma<64, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
@@ -321,6 +421,139 @@ bitnet_status bitnet_i2s_quant_gemv(const uint8_t* packed, int64_t N, int64_t K,
   if (e != cudaSuccess) return cuda_fail(e, "launch of the activation quant kernel");
   st = run_matmul(packed, N, K, xq, xs, M, Y, acc_or_null, true, s, dev);
   return st == BITNET_OK ? ok() : st;
+}
+
+size_t bitnet_i2s_quant_gemv_batched_workspace_bytes(const bitnet_i2s_problem* problems,
+                                                     int count, int64_t M) {
+  if (problems == nullptr || count < 1 || M < 1) return 0;
+  size_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    const size_t one = bitnet_i2s_quant_gemv_workspace_bytes(M, problems[i].K);
+    if (one == 0) return 0;
+    total += one;
+  }
+  return total;
+}
+
+bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, int count,
+                                            int64_t M, void* workspace, size_t workspace_bytes,
+                                            void* stream) {
+  if (problems == nullptr || count < 1)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_quant_gemv_batched: no problems");
+  if (M < 1 || M > kMaxTokens)
+    return fail(BITNET_ERR_SHAPE, "bitnet_i2s_quant_gemv_batched: M=%lld", (long long)M);
+  int64_t kmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_i2s_problem& q = problems[i];
+    bitnet_status st = check_matmul_args("bitnet_i2s_quant_gemv_batched", q.packed, q.N, q.K, q.X,
+                                         q.X, M, q.Y, kMaxTokens);
+    if (st != BITNET_OK) return st;
+    kmax = std::max(kmax, q.K);
+  }
+  if (workspace == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_quant_gemv_batched: null workspace");
+  if (!aligned(workspace, 256))
+    return fail(BITNET_ERR_ALIGN,
+                "bitnet_i2s_quant_gemv_batched: workspace must be 256-byte aligned");
+  const size_t need = bitnet_i2s_quant_gemv_batched_workspace_bytes(problems, count, M);
+  if (workspace_bytes < need)
+    return fail(BITNET_ERR_INVALID_ARG,
+                "bitnet_i2s_quant_gemv_batched: workspace of %zu bytes < %zu", workspace_bytes,
+                need);
+  int dev;
+  bitnet_status st = check_device(&dev);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool dp4a = use_dp4a(M, kmax);
+  static thread_local BatchParamsT<kMaxBatch> bp;  // 16 KB: kept off the stack
+  for (int base = 0; base < count; base += kMaxBatch) {
+    const int cnt = std::min(kMaxBatch, count - base);
+    bp.count = cnt;
+    bp.m = static_cast<int32_t>(M);
+    for (int i = 0; i < cnt; ++i) {
+      const bitnet_i2s_problem& q = problems[base + i];
+      int8_t* xq = reinterpret_cast<int8_t*>(ws);
+      float* xs = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(M) * q.K));
+      ws += bitnet_i2s_quant_gemv_workspace_bytes(M, q.K);
+      bp.p[i] = make_problem(q.packed, q.N, q.K, q.X, xq, xs, q.Y, q.acc_or_null);
+    }
+    if (dp4a) {
+      // One launch quantizes every problem's tokens, one launch does every
+      // matmul; the second is a dependent launch of the first.
+      cudaLaunchConfig_t cfg;
+      std::memset(&cfg, 0, sizeof(cfg));
+      cfg.gridDim = dim3(static_cast<unsigned>(cnt * M));
+      cfg.blockDim = dim3(256);
+      cfg.stream = s;
+      cudaLaunchAttribute attr = pdl_attr(true);
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_batched_kernel<kMaxBatch>, bp);
+      if (e != cudaSuccess) return cuda_fail(e, "launch of the batched activation quant kernel");
+      st = launch_dp4a(bp, s, true, dev);
+      if (st != BITNET_OK) return st;
+    } else {
+      for (int i = 0; i < cnt; ++i) {
+        const BatchProblem& q = bp.p[i];
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(static_cast<unsigned>(M));
+        cfg.blockDim = dim3(256);
+        cfg.stream = s;
+        cudaLaunchAttribute attr = pdl_attr(true);
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, q.x, static_cast<int64_t>(q.k),
+                                           q.xq, q.xs);
+        if (e != cudaSuccess) return cuda_fail(e, "launch of the activation quant kernel");
+        st = run_matmul(q.packed, q.n, q.k, q.xq, q.xs, M, q.y, q.acc, true, s, dev);
+        if (st != BITNET_OK) return st;
+      }
+    }
+  }
+  return ok();
+}
+
+bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int count, int64_t M,
+                                      void* stream) {
+  if (problems == nullptr || count < 1)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_gemv_batched: no problems");
+  if (M < 1 || M > kMaxTokens)
+    return fail(BITNET_ERR_SHAPE, "bitnet_i2s_gemv_batched: M=%lld", (long long)M);
+  int64_t kmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_i2s_qproblem& q = problems[i];
+    bitnet_status st = check_matmul_args("bitnet_i2s_gemv_batched", q.packed, q.N, q.K, q.Xq,
+                                         q.xs, M, q.Y, kMaxTokens);
+    if (st != BITNET_OK) return st;
+    kmax = std::max(kmax, q.K);
+  }
+  int dev;
+  bitnet_status st = check_device(&dev);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!use_dp4a(M, kmax)) {
+    for (int i = 0; i < count; ++i) {
+      const bitnet_i2s_qproblem& q = problems[i];
+      st = run_matmul(q.packed, q.N, q.K, q.Xq, q.xs, M, q.Y, q.acc_or_null, false, s, dev);
+      if (st != BITNET_OK) return st;
+    }
+    return ok();
+  }
+  static thread_local BatchParamsT<kMaxBatch> bp;
+  for (int base = 0; base < count; base += kMaxBatch) {
+    const int cnt = std::min(kMaxBatch, count - base);
+    bp.count = cnt;
+    bp.m = static_cast<int32_t>(M);
+    for (int i = 0; i < cnt; ++i) {
+      const bitnet_i2s_qproblem& q = problems[base + i];
+      bp.p[i] = make_problem(q.packed, q.N, q.K, nullptr, q.Xq, q.xs, q.Y, q.acc_or_null);
+    }
+    st = launch_dp4a(bp, s, false, dev);
+    if (st != BITNET_OK) return st;
+  }
+  return ok();
 }
 
 bitnet_status bitnet_device_status(void) {

@@ -80,21 +80,16 @@ __global__ void __launch_bounds__(256) i2s_pack_kernel(const float* __restrict__
 }
 
 // ------------------------------------------------------ activation quant
-// One CTA per token row: amax over the row, then xq = clamp(rint(x*127/amax))
+// One token row: amax over the row, then xq = clamp(rint(x*127/amax))
 // ["LLM Quantization Paradigms ...", section 5, The Mathematics of BitNet
 // b1.58: per-token AbsMax to 8 bits].  Division and multiplication are the
 // IEEE round-to-nearest operations and the rounding to integer is half to
-// even, so the codes are a deterministic function of the inputs.
-// With PDL the kernel first waits for the preceding grid, then lets the
-// dependent grid (the matmul) launch and start streaming its weights.
-__global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict__ x, int64_t k,
-                                                        int8_t* __restrict__ xq,
-                                                        float* __restrict__ xs) {
-  grid_dependency_wait();
-  grid_dependents_launch();
-  __shared__ float red[32];
-  const int64_t row = blockIdx.x;
-  const float4* xr = reinterpret_cast<const float4*>(x + row * k);
+// even, so the codes are a deterministic function of the inputs.  Called by
+// every thread of the CTA; k is a multiple of 16.
+__device__ __forceinline__ void quantize_row(const float* __restrict__ xrow, int64_t k,
+                                             int8_t* __restrict__ qrow, float* __restrict__ xs_out,
+                                             float* red) {
+  const float4* xr = reinterpret_cast<const float4*>(xrow);
   const int64_t k4 = k >> 2;
   float m = 0.0f;
   for (int64_t i = threadIdx.x; i < k4; i += blockDim.x) {
@@ -103,7 +98,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict_
   }
   const float amax = block_max_nonneg(m, red);
   const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-  char4* out = reinterpret_cast<char4*>(xq + row * k);
+  char4* out = reinterpret_cast<char4*>(qrow);
   for (int64_t i = threadIdx.x; i < k4; i += blockDim.x) {
     const float4 v = xr[i];
     char4 q;
@@ -113,7 +108,20 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict_
     q.w = static_cast<signed char>(max(-127, min(127, __float2int_rn(__fmul_rn(v.w, inv)))));
     out[i] = q;
   }
-  if (threadIdx.x == 0) xs[row] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+  if (threadIdx.x == 0) *xs_out = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+}
+
+// One CTA per token row.  With PDL the kernel first waits for the preceding
+// grid, then lets the dependent grid (the matmul) launch and start streaming
+// its weights.
+__global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict__ x, int64_t k,
+                                                        int8_t* __restrict__ xq,
+                                                        float* __restrict__ xs) {
+  grid_dependency_wait();
+  grid_dependents_launch();
+  __shared__ float red[32];
+  const int64_t row = blockIdx.x;
+  quantize_row(x + row * k, k, xq + row * k, xs + row, red);
 }
 
 }  // namespace bitnet

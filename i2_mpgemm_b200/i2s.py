@@ -38,6 +38,9 @@ SIGNATURES = {
     "bitnet_i2s_gemm": (_I32, [_VP, _I64, _I64, _VP, _VP, _I64, _VP, _VP, _VP]),
     "bitnet_i2s_quant_gemv_workspace_bytes": (_SZ, [_I64, _I64]),
     "bitnet_i2s_quant_gemv": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
+    "bitnet_i2s_quant_gemv_batched_workspace_bytes": (_SZ, [_VP, _I32, _I64]),
+    "bitnet_i2s_quant_gemv_batched": (_I32, [_VP, _I32, _I64, _VP, _SZ, _VP]),
+    "bitnet_i2s_gemv_batched": (_I32, [_VP, _I32, _I64, _VP]),
     "bitnet_device_status": (_I32, []),
     "bitnet_last_error": (ctypes.c_char_p, []),
 }
@@ -172,6 +175,92 @@ def bitnet_i2s_quant_gemv(packed, n, k, x, y=None, acc=None, workspace=None, wan
     _check(lib.bitnet_i2s_quant_gemv(_ptr(packed), n, k, _ptr(x), m, _ptr(y), _ptr(acc),
                                      _ptr(workspace), workspace.numel(), _stream(stream)))
     return (y, acc) if acc is not None else y
+
+
+class Problem(ctypes.Structure):
+    """ctypes mirror of `bitnet_i2s_problem`."""
+    _fields_ = [("packed", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("X", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("acc_or_null", ctypes.c_void_p)]
+
+
+class BatchedQuantGemv:
+    """Argument block of one bitnet_i2s_quant_gemv_batched call.
+
+    `problems` is a list of (packed, N, K, X, Y, acc_or_None) with CUDA
+    tensors; every X has M rows.  The descriptor array and the workspace are
+    built once, so `run()` (capturable in a CUDA graph) only makes the call.
+    """
+
+    def __init__(self, problems, m: int, workspace: torch.Tensor | None = None):
+        self.m = int(m)
+        self.tensors = []  # keep every tensor alive as long as the descriptors
+        arr = (Problem * len(problems))()
+        for i, (packed, n, k, x, y, acc) in enumerate(problems):
+            _need(packed, "packed", torch.uint8, bitnet_i2s_packed_bytes(n, k))
+            _need(x, "X", torch.float32, self.m * k)
+            _need(y, "Y", torch.float32, self.m * n)
+            if acc is not None:
+                _need(acc, "acc", torch.int32, self.m * n)
+            arr[i] = Problem(packed.data_ptr(), n, k, x.data_ptr(), y.data_ptr(),
+                             None if acc is None else acc.data_ptr())
+            self.tensors += [packed, x, y, acc]
+        self.array = arr
+        self.count = len(problems)
+        need = int(lib.bitnet_i2s_quant_gemv_batched_workspace_bytes(arr, self.count, self.m))
+        if need == 0:
+            raise BitnetError(1, "invalid batch")
+        if workspace is None:
+            dev = problems[0][0].device
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _need(workspace, "workspace", torch.uint8, need)
+        self.workspace = workspace
+
+    def run(self, stream=None) -> None:
+        _check(lib.bitnet_i2s_quant_gemv_batched(self.array, self.count, self.m,
+                                                 self.workspace.data_ptr(),
+                                                 self.workspace.numel(), _stream(stream)))
+
+
+def bitnet_i2s_quant_gemv_batched(problems, m: int, workspace=None, stream=None) -> None:
+    """One call for many independent (packed, N, K, X, Y, acc) problems."""
+    BatchedQuantGemv(problems, m, workspace).run(stream)
+
+
+class QProblem(ctypes.Structure):
+    """ctypes mirror of `bitnet_i2s_qproblem`."""
+    _fields_ = [("packed", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("Xq", ctypes.c_void_p), ("xs", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+                ("acc_or_null", ctypes.c_void_p)]
+
+
+class BatchedGemv:
+    """Argument block of one bitnet_i2s_gemv_batched call: a list of
+    (packed, N, K, Xq, xs, Y, acc_or_None) CUDA tensors, every Xq with M rows."""
+
+    def __init__(self, problems, m: int):
+        self.m = int(m)
+        self.tensors = []
+        arr = (QProblem * len(problems))()
+        for i, (packed, n, k, xq, xs, y, acc) in enumerate(problems):
+            _need(packed, "packed", torch.uint8, bitnet_i2s_packed_bytes(n, k))
+            _need(xq, "Xq", torch.int8, self.m * k)
+            _need(xs, "xs", torch.float32, self.m)
+            _need(y, "Y", torch.float32, self.m * n)
+            if acc is not None:
+                _need(acc, "acc", torch.int32, self.m * n)
+            arr[i] = QProblem(packed.data_ptr(), n, k, xq.data_ptr(), xs.data_ptr(), y.data_ptr(),
+                              None if acc is None else acc.data_ptr())
+            self.tensors += [packed, xq, xs, y, acc]
+        self.array = arr
+        self.count = len(problems)
+
+    def run(self, stream=None) -> None:
+        _check(lib.bitnet_i2s_gemv_batched(self.array, self.count, self.m, _stream(stream)))
+
+
+def bitnet_i2s_gemv_batched(problems, m: int, stream=None) -> None:
+    """One call for many independent (packed, N, K, Xq, xs, Y, acc) problems."""
+    BatchedGemv(problems, m).run(stream)
 
 
 def bitnet_device_status() -> None:

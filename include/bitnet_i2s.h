@@ -133,6 +133,57 @@ BITNET_API bitnet_status bitnet_i2s_quant_gemv(const uint8_t* packed, int64_t N,
                                     int64_t M, float* Y, int32_t* acc_or_null, void* workspace,
                                     size_t workspace_bytes, void* stream);
 
+/* One independent problem of a batched call (device pointers; layouts as for
+ * bitnet_i2s_quant_gemv): Y[M,N] = matmul(I2_S W[N,K], quant(X[M,K])). */
+typedef struct bitnet_i2s_problem {
+  const uint8_t* packed;  /* I2_S tensor, 16-byte aligned */
+  int64_t N;
+  int64_t K;              /* multiple of 128 */
+  const float* X;         /* M*K fp32, 16-byte aligned */
+  float* Y;               /* M*N fp32 */
+  int32_t* acc_or_null;   /* M*N int32 or NULL */
+} bitnet_i2s_problem;
+
+/* Workspace bytes bitnet_i2s_quant_gemv_batched needs (0 for bad arguments). */
+BITNET_API size_t bitnet_i2s_quant_gemv_batched_workspace_bytes(const bitnet_i2s_problem* problems,
+                                                                int count, int64_t M);
+
+/* bitnet_i2s_quant_gemv for `count` independent problems that share the token
+ * count M, as few launches as possible: for M <= 2 (K <= 8192) one launch
+ * quantizes every problem's activations and one persistent launch streams
+ * every problem's packed weights, so the whole batch (for example the 210
+ * projections of a 30-layer BitNet b1.58 stack) keeps HBM busy end to end.
+ * Results are identical to calling bitnet_i2s_quant_gemv on each problem
+ * [P5 section 5: per-token AbsMax quantization, then the ternary contraction].
+ *   problems: HOST array of `count` descriptors, read during the call only.
+ *   workspace: device scratch of at least
+ *     bitnet_i2s_quant_gemv_batched_workspace_bytes(problems, count, M) bytes,
+ *     256-byte aligned, not shared with work that may run at the same time.
+ * The problems' outputs must not overlap each other or any input. */
+BITNET_API bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, int count,
+                                                       int64_t M, void* workspace,
+                                                       size_t workspace_bytes, void* stream);
+
+/* One problem of bitnet_i2s_gemv_batched: activations already quantized. */
+typedef struct bitnet_i2s_qproblem {
+  const uint8_t* packed;  /* I2_S tensor, 16-byte aligned */
+  int64_t N;
+  int64_t K;              /* multiple of 128 */
+  const int8_t* Xq;       /* M*K int8, 16-byte aligned */
+  const float* xs;        /* M fp32 */
+  float* Y;               /* M*N fp32 */
+  int32_t* acc_or_null;   /* M*N int32 or NULL */
+} bitnet_i2s_qproblem;
+
+/* bitnet_i2s_gemm on `count` independent problems sharing the token count M
+ * (for example q, k and v on one quantized input), in one persistent launch
+ * when M <= 2 and every K <= 8192, else one launch per problem.  Same
+ * results as the single-problem call [P5 section 5 figure; P1 "How I2_S
+ * Kernels Process the Format"].  `problems` is a HOST array read during the
+ * call only; no workspace is needed. */
+BITNET_API bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int count,
+                                                 int64_t M, void* stream);
+
 /* Waits for all work on the current device, then returns
  * BITNET_ERR_DEVICE_TIMEOUT if any kernel of this library gave up on a
  * bounded wait since the last call (and clears the flag), BITNET_ERR_CUDA if

@@ -272,3 +272,104 @@ def test_large_layer_sampled(i2s, m):
 
 def test_no_device_wait_timed_out(i2s):
     i2s.bitnet_device_status()
+
+
+# ------------------------------------------- decode ALU path and batching
+
+# M = 1, 2 with K <= 8192 run on the integer-ALU decode kernel.
+DECODE = [(1, 1, 128), (1, 300, 2560), (2, 130, 640), (1, 129, 8192), (2, 257, 8192),
+          (2, 64, 4096), (1, 1000, 6912), (2, 7, 384)]
+
+
+@pytest.mark.parametrize("m,n,k", DECODE)
+def test_decode_alu_path_matches_oracle(i2s, m, n, k):
+    w, t, x, packed, xq, xs = _case(m, n, k, 17 * m + 3 * n + k)
+    y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+    d_packed = dev(torch.from_numpy(packed))
+    y, acc = i2s.bitnet_i2s_gemv(d_packed, n, k, dev(torch.from_numpy(xq)),
+                                 dev(torch.from_numpy(xs)), want_acc=True)
+    assert_acc_equal(acc.cpu().numpy(), acc_ref, "gemv")
+    assert_y_close(y.cpu().numpy(), y_ref, "gemv")
+    y, acc = i2s.bitnet_i2s_quant_gemv(d_packed, n, k, dev(x), want_acc=True)
+    assert_acc_equal(acc.cpu().numpy(), acc_ref, "quant_gemv")
+    assert_y_close(y.cpu().numpy(), y_ref, "quant_gemv")
+
+
+def _batched_problems(shapes, m, seed):
+    cases, problems = [], []
+    for i, (n, k) in enumerate(shapes):
+        w, t, x, packed, xq, xs = _case(m, n, k, seed + i)
+        d_packed, d_x = dev(torch.from_numpy(packed)), dev(x)
+        y = torch.empty((m, n), device="cuda")
+        acc = torch.empty((m, n), dtype=torch.int32, device="cuda")
+        problems.append((d_packed, n, k, d_x, y, acc))
+        cases.append((packed, n, k, xq, xs))
+    return cases, problems
+
+
+@pytest.mark.parametrize("m", [1, 2, 4, 70])
+def test_batched_mixed_shapes(i2s, m):
+    shapes = [(7, 128), (300, 640), (130, 2560), (64, 6912), (1, 384), (257, 1024)]
+    cases, problems = _batched_problems(shapes, m, 900 + m)
+    i2s.bitnet_i2s_quant_gemv_batched(problems, m)
+    for (packed, n, k, xq, xs), (_, _, _, _, y, acc) in zip(cases, problems):
+        y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+        assert_acc_equal(acc.cpu().numpy(), acc_ref, f"{n}x{k}")
+        assert_y_close(y.cpu().numpy(), y_ref, f"{n}x{k}")
+
+
+def test_batched_more_than_one_launch_worth_of_problems(i2s):
+    shapes = [(3 + (i % 5), 128 * (1 + i % 3)) for i in range(300)]
+    cases, problems = _batched_problems(shapes, 1, 4000)
+    plan = i2s.BatchedQuantGemv(problems, 1)
+    plan.run()
+    plan.run()  # a second call on the same workspace gives the same results
+    for (packed, n, k, xq, xs), (_, _, _, _, y, acc) in zip(cases, problems):
+        y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+        assert_acc_equal(acc.cpu().numpy(), acc_ref)
+        assert_y_close(y.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("m", [1, 2, 16])
+def test_stack_batched_all_layers_sampled(i2s, m):
+    """The 210-projection stack through one batched call, as the benchmark runs it."""
+    problems, keep = [], []
+    for layer in range(inputs.LAYERS_2B):
+        for idx, p in enumerate(inputs.projections_2b()):
+            seed = inputs.seed_stack(layer, idx)
+            w, t, s = inputs.ternary_weights(p.n, p.k, seed)
+            x = inputs.activations(m, p.k, seed)
+            packed = oracle.pack(w.numpy())
+            d_packed = dev(torch.from_numpy(packed))
+            y = torch.empty((m, p.n), device="cuda")
+            acc = torch.empty((m, p.n), dtype=torch.int32, device="cuda")
+            problems.append((d_packed, p.n, p.k, dev(x), y, acc))
+            keep.append((packed, p.n, p.k, x, t, seed))
+    i2s.bitnet_i2s_quant_gemv_batched(problems, m)
+    torch.cuda.synchronize()
+    for (packed, n, k, x, t, seed), (_, _, _, _, y, acc) in zip(keep, problems):
+        xq, xs = oracle.act_quant(x.numpy())
+        pm, pn = sample_positions(m, n, 32, seed)
+        y_ref, acc_ref = oracle.gemm_sampled(packed, n, k, xq, xs, pm, pn)
+        acc_h = acc.cpu()
+        assert_acc_equal(acc_h.numpy()[pm, pn], acc_ref, f"{n}x{k}")
+        assert_y_close(y.cpu().numpy()[pm, pn], y_ref, f"{n}x{k}")
+        assert column_sum_identity(acc_h, torch.from_numpy(xq), t)
+
+
+@pytest.mark.parametrize("m", [1, 2, 5])
+def test_gemv_batched_on_quantized_inputs(i2s, m):
+    shapes = [(640, 2560), (640, 2560), (2560, 2560), (33, 6912), (130, 128)]
+    cases, problems = [], []
+    for i, (n, k) in enumerate(shapes):
+        w, t, x, packed, xq, xs = _case(m, n, k, 7000 + i)
+        y = torch.empty((m, n), device="cuda")
+        acc = torch.empty((m, n), dtype=torch.int32, device="cuda")
+        problems.append((dev(torch.from_numpy(packed)), n, k, dev(torch.from_numpy(xq)),
+                         dev(torch.from_numpy(xs)), y, acc))
+        cases.append((packed, n, k, xq, xs))
+    i2s.bitnet_i2s_gemv_batched(problems, m)
+    for (packed, n, k, xq, xs), pr in zip(cases, problems):
+        y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+        assert_acc_equal(pr[6].cpu().numpy(), acc_ref)
+        assert_y_close(pr[5].cpu().numpy(), y_ref)
