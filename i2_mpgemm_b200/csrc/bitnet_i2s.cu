@@ -192,38 +192,38 @@ int sm_count(int dev) {
 }
 
 // The integer-ALU kernel serves one or two tokens with K up to 8192 (the
-// activations of one problem live in registers); everything else goes to the
-// tensor-core kernel.
-constexpr int64_t kDp4aMaxK = 8192;
-bool use_dp4a(int64_t m, int64_t kmax) { return m >= 1 && m <= 2 && kmax <= kDp4aMaxK; }
+// activations of one problem sit in a shared-memory slot); everything else
+// goes to the tensor-core kernel.
+constexpr int kMaxBatch = 160;  // problems per launch: the parameter block stays under 32 KB
+bool use_dp4a(int64_t m, int64_t kmax) { return m >= 1 && m <= 2 && kmax <= kGemvMaxK; }
 
-// Split every problem into work items of consecutive rows: about one item
-// per SM over the whole batch, never more than one 32 KB stage per item.
+// Tensor maps, 128-row tiles and their stage counts for every problem.
 template <int CAP>
-bitnet_status plan_items(BatchParamsT<CAP>& bp, int sms) {
-  int64_t total_rows = 0;
-  for (int i = 0; i < bp.count; ++i) total_rows += bp.p[i].n;
-  const int64_t target = std::max<int64_t>(1, (total_rows + sms - 1) / sms);
-  int64_t items = 0;
+bitnet_status plan_items(BatchParamsT<CAP>& bp) {
+  int64_t items = 0, stages = 0;
   for (int i = 0; i < bp.count; ++i) {
     BatchProblem& q = bp.p[i];
-    const int64_t cap = std::max<int64_t>(1, 32768 / (q.k / 4));
-    const int64_t rpi = std::min(target, cap);
-    q.rows_per_item = static_cast<int32_t>(rpi);
+    bitnet_status st = encode_u8_2d(&bp.tmap[i], q.packed, static_cast<uint64_t>(q.k / 4),
+                                    static_cast<uint64_t>(q.n), 128, kGemvTileRows);
+    if (st != BITNET_OK) return st;
     q.item_start = static_cast<int32_t>(items);
-    items += (q.n + rpi - 1) / rpi;
-    if (items > int64_t{0x7fffffff}) return fail(BITNET_ERR_SHAPE, "too many rows in one batch");
+    q.stage_start = static_cast<int32_t>(stages);
+    const int64_t tiles = (q.n + kGemvTileRows - 1) / kGemvTileRows;
+    items += tiles;
+    stages += tiles * ((q.k + 511) / 512);
+    if (stages > int64_t{0x7fffffff}) return fail(BITNET_ERR_SHAPE, "too many rows in one batch");
   }
   bp.total_items = static_cast<int32_t>(items);
+  bp.total_stages = static_cast<int32_t>(stages);
   return BITNET_OK;
 }
 
-template <int MT, int WPL, int CAP>
+template <int MT, int CAP>
 bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, int grid, cudaStream_t stream, bool pdl,
                             int dev) {
-  using C = GemvCfg<MT, WPL>;
+  using C = GemvCfg<MT>;
   static std::atomic<uint8_t> smem_done[kMaxDevices];
-  auto kern = i2s_gemv_dp4a_kernel<MT, WPL, CAP>;
+  auto kern = i2s_gemv_dp4a_kernel<MT, CAP>;
   bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
   if (st != BITNET_OK) return st;
   cudaLaunchConfig_t cfg;
@@ -240,20 +240,15 @@ bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, int grid, cudaStream_t 
   return BITNET_OK;
 }
 
+// Persistent grid: two CTAs per SM, never more CTAs than row tiles.
 template <int CAP>
 bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev) {
-  const int sms = sm_count(dev);
-  bitnet_status st = plan_items(bp, sms);
+  bitnet_status st = plan_items(bp);
   if (st != BITNET_OK) return st;
-  int kmax = 0;
-  for (int i = 0; i < bp.count; ++i) kmax = std::max(kmax, bp.p[i].k);
   bp.pdl = pdl ? 1 : 0;
-  const int grid = std::min(bp.total_items, sms);
-  if (bp.m == 1)
-    return kmax <= 4096 ? launch_dp4a_t<1, 8, CAP>(bp, grid, stream, pdl, dev)
-                        : launch_dp4a_t<1, 16, CAP>(bp, grid, stream, pdl, dev);
-  return kmax <= 4096 ? launch_dp4a_t<2, 8, CAP>(bp, grid, stream, pdl, dev)
-                      : launch_dp4a_t<2, 16, CAP>(bp, grid, stream, pdl, dev);
+  const int grid = std::min(bp.total_items, 2 * sm_count(dev));
+  return bp.m == 1 ? launch_dp4a_t<1, CAP>(bp, grid, stream, pdl, dev)
+                   : launch_dp4a_t<2, CAP>(bp, grid, stream, pdl, dev);
 }
 
 BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const float* x,
@@ -267,8 +262,8 @@ BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const flo
   q.acc = acc;
   q.n = static_cast<int32_t>(n);
   q.k = static_cast<int32_t>(k);
-  q.rows_per_item = 0;
   q.item_start = 0;
+  q.stage_start = 0;
   return q;
 }
 
@@ -466,7 +461,7 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const bool dp4a = use_dp4a(M, kmax);
-  static thread_local BatchParamsT<kMaxBatch> bp;  // 16 KB: kept off the stack
+  static thread_local BatchParamsT<kMaxBatch> bp;  // 30 KB: kept off the stack
   for (int base = 0; base < count; base += kMaxBatch) {
     const int cnt = std::min(kMaxBatch, count - base);
     bp.count = cnt;

@@ -4,33 +4,33 @@
 // At one or two tokens the ternary contraction ("LLM Quantization
 // Paradigms: FP8, AWQ, EXL2 & BitNet b1.58 in 2026", section 5 figure,
 // "BitNet b1.58 Ternary Matrix Multiplication") does 4 multiply-adds per
-// packed byte per token, far below what the SM's dp4a pipe sustains at HBM
-// speed, so it runs as dp4a on registers while the packed weights stream
-// through shared memory:
+// packed byte per token, well within what dp4a sustains at HBM speed, so it
+// runs on the ALU while the packed weights stream through shared memory:
 //
-//   * Work item = a group of consecutive rows of one problem.  Rows of the
-//     I2_S tensor are contiguous, so a group is one contiguous byte range
-//     fetched with one 1-D bulk copy into a shared-memory stage.
-//   * Each CTA owns one contiguous range of items (items have about the
-//     same byte count, so equal ranges balance), so it switches problem only
-//     a few times per launch.
-//   * Warp 0 (one lane) is the producer: it walks the CTA's items, keeps
-//     kStages copies in flight, and when an item starts a new problem it
-//     also copies that problem's int8 activations (M x K bytes) into one of
-//     two x slots and stages the problem's scales next to them.
-//   * Warps 1..12 (1..8 for two tokens) compute, two rows at a time per
-//     warp (two independent dependency chains).  Lane l owns packed words l, l+32, ... of every
-//     row (so its loads of a row are conflict-free and coalesced) and holds
-//     the matching activation words in registers for the whole problem.
+//   * Work item = a tile of 128 rows of one problem over the whole K.
+//     The tile streams in stages of one TMA box of 128 rows x 128 bytes
+//     (512 weights of each row) written with the 128-byte swizzle.
+//   * Each CTA owns one contiguous range of items, balanced by bytes, so it
+//     changes problem only a few times per launch.  Warp 0 (one lane) is the
+//     producer; on a change of problem it also copies the problem's int8
+//     activations (M x K bytes) into one of two x slots and stages the two
+//     scales next to them.
+//   * Warps 1..4 compute.  Lane l of warp w owns row 32w + l of the tile:
+//     it reads its row 16 bytes at a time (the swizzle makes the 8 lanes of
+//     each quarter-warp hit 8 different bank groups) and keeps int32
+//     accumulators for its row only, so no cross-lane reduction is needed
+//     and the tile's outputs are stored coalesced.  All lanes need the same
+//     activation bytes at the same time: those are 16-byte broadcast loads.
 //
 // Unpack without shifts ("How BitNet's 1-Bit (I2_S) Quantization Works
 // Compared to Standard LLM Quantization", Ternary Representation and
 // Packing: group g of a byte is bits [7-2g : 6-2g]): word & (3 << (6-2g)) in
-// every byte is code_g * 4^(3-g), an unsigned byte in {0, 4^(3-g), 2*4^(3-g)}.
-// One dp4a per group and token accumulates sum code*x scaled by 4^(3-g) in
-// its own register; at the end of the row the four are rescaled exactly
-// (arithmetic shifts of exact multiples), summed, reduced over the warp,
-// and sum_k x is subtracted, since w = code - 1.
+// every byte is code_g * 4^(3-g), an unsigned byte.  One dp4a per group,
+// word and token accumulates sum code*x scaled by 4^(3-g) in its own
+// register; the four are rescaled exactly (arithmetic shifts of exact
+// multiples) and summed at the end of the tile, and sum_k x is subtracted
+// because w = code - 1.  Bytes of a box past K read as zero, i.e. code 0,
+// and contribute nothing.
 #pragma once
 
 #include "ptx.cuh"
@@ -38,9 +38,10 @@
 
 namespace bitnet {
 
-constexpr int kMaxBatch = 256;
+constexpr int kGemvTileRows = 128;
+constexpr int kGemvMaxK = 8192;  // the x slot holds M x K bytes, K <= 8192
 
-// One independent problem of a batch (all device pointers).
+// One independent problem of a batch (device pointers and shape).
 struct BatchProblem {
   const uint8_t* packed;  // I2_S tensor [n, k]
   const float* x;         // fp32 activations [m, k] (read by the batched quantizer)
@@ -49,37 +50,41 @@ struct BatchProblem {
   float* y;               // [m, n]
   int32_t* acc;           // [m, n] or null
   int32_t n, k;
-  int32_t rows_per_item;  // rows of one work item
-  int32_t item_start;     // first global work item of this problem
+  int32_t item_start;     // first global work item (row tile) of this problem
+  int32_t stage_start;    // first global stage (one box each) of this problem
 };
 
 template <int CAP>
 struct BatchParamsT {
-  int32_t count;        // problems
-  int32_t m;            // tokens (the same for every problem)
-  int32_t total_items;  // work items over all problems
-  int32_t pdl;          // 1: activations come from the preceding grid
+  int32_t count;         // problems
+  int32_t m;             // tokens (the same for every problem)
+  int32_t total_items;   // row tiles over all problems
+  int32_t total_stages;  // boxes over all problems
+  int32_t pdl;           // 1: activations come from the preceding grid
+  int32_t pad[11];
+  CUtensorMap tmap[CAP];  // per problem: packed bytes as [n rows, k/4 bytes], box 128 x 128
   BatchProblem p[CAP];
 };
 
 struct StageMeta {
-  int32_t p, row0, nrows, sw;  // sw: index of the problem switch this item starts, or -1
+  int32_t p;     // problem
+  int32_t row0;  // first row of the tile
+  int32_t kc;    // box index along K (512 weights each)
+  int32_t info;  // bit 0: first box of the tile, bit 1: last box, bits 8..: switch index + 1
 };
 
-template <int MT, int WPL>
+template <int MT>
 struct GemvCfg {
   static_assert(MT >= 1 && MT <= 2, "tokens");
-  static constexpr int kComputeWarps = MT == 1 ? 12 : 8;
-  static constexpr int kRowsPerPass = 2;  // rows one warp interleaves
+  static constexpr int kComputeWarps = kGemvTileRows / 32;
   static constexpr int kThreads = 32 * (kComputeWarps + 1);
-  static constexpr int kStageBytes = 32768;
+  static constexpr int kBoxBytes = kGemvTileRows * 128;  // 16 KB
   static constexpr int kStages = 4;
-  static constexpr int kMaxK = WPL * 512;  // 32 lanes x WPL words x 16 weights
-  static constexpr int kXSlotBytes = MT * kMaxK;
+  static constexpr int kXSlotBytes = MT * kGemvMaxK + 512;  // + slack read past K, never used
   static constexpr int kBars = 2 * kStages + 4;
-  static constexpr size_t kSmemBytes = 128 + static_cast<size_t>(kStages) * kStageBytes +
-                                       2 * kXSlotBytes + kBars * 8 + kStages * sizeof(StageMeta) +
-                                       2 * 4 * sizeof(float) + 16;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kBoxBytes +
+                                       2 * kXSlotBytes + kBars * 8 +
+                                       kStages * sizeof(StageMeta) + 2 * 4 * sizeof(float) + 16;
 };
 
 __device__ __forceinline__ int dp4a_u8s8(uint32_t a, uint32_t b, int c) {
@@ -89,7 +94,7 @@ __device__ __forceinline__ int dp4a_u8s8(uint32_t a, uint32_t b, int c) {
 }
 
 template <typename BP>
-__device__ __forceinline__ int find_problem(const BP& bp, int item) {
+__device__ __forceinline__ int find_problem_by_item(const BP& bp, int item) {
   int lo = 0, hi = bp.count - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -99,19 +104,37 @@ __device__ __forceinline__ int find_problem(const BP& bp, int item) {
   return lo;
 }
 
-template <int MT, int WPL, int CAP>
-__global__ void __launch_bounds__(GemvCfg<MT, WPL>::kThreads, 1)
+// First item whose first stage is at or after global stage `target`; items
+// of one problem all have ceil(k/512) stages.
+template <typename BP>
+__device__ __forceinline__ int first_item_at_stage(const BP& bp, int target) {
+  if (target >= bp.total_stages) return bp.total_items;
+  int lo = 0, hi = bp.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (bp.p[mid].stage_start <= target) lo = mid;
+    else hi = mid - 1;
+  }
+  const BatchProblem& P = bp.p[lo];
+  const int nk = (P.k + 511) >> 9;
+  const int items = (P.n + kGemvTileRows - 1) / kGemvTileRows;
+  const int off = (target - P.stage_start + nk - 1) / nk;
+  return off >= items ? P.item_start + items : P.item_start + off;
+}
+
+template <int MT, int CAP>
+__global__ void __launch_bounds__(GemvCfg<MT>::kThreads, 2)
     i2s_gemv_dp4a_kernel(const __grid_constant__ BatchParamsT<CAP> bp) {
-  using C = GemvCfg<MT, WPL>;
+  using C = GemvCfg<MT>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
-  uint8_t* stages = smem;
-  uint8_t* xslots = smem + S * C::kStageBytes;
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* boxes = smem;
+  uint8_t* xslots = smem + S * C::kBoxBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(xslots + 2 * C::kXSlotBytes);
   StageMeta* meta = reinterpret_cast<StageMeta*>(bars + C::kBars);
-  float* xscal = reinterpret_cast<float*>(meta + S);  // per x slot: weight scale, xs[0..MT)
+  float* xscal = reinterpret_cast<float*>(meta + S);  // per slot: weight scale, xs[0..MT)
   volatile uint32_t* abort_flag = reinterpret_cast<uint32_t*>(xscal + 8);
 
   const int warp = threadIdx.x >> 5;
@@ -136,92 +159,103 @@ __global__ void __launch_bounds__(GemvCfg<MT, WPL>::kThreads, 1)
   }
   __syncthreads();
 
-  const int total = bp.total_items;
   const int m_tokens = bp.m;
-  const int item_lo = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
-  const int item_hi = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
+  const int64_t ts = bp.total_stages;
+  const int item_lo = first_item_at_stage(bp, static_cast<int>(ts * blockIdx.x / gridDim.x));
+  const int item_hi = first_item_at_stage(bp, static_cast<int>(ts * (blockIdx.x + 1) / gridDim.x));
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      // Weights of the first stages do not depend on the preceding grid:
-      // request them before waiting for it.
-      // Per stage: the last item whose copy was issued, and whether its
-      // phase has received the producer's arrival.
-      int issued_item[S];
-      bool issued_arrived[S];
+      int issued = 0;    // boxes issued
+      int nsw = 0;       // problem switches announced to the consumers
+      int x_loaded = 0;  // switches whose activations were requested
+      int prev_p = -1;
+      bool waited = (bp.pdl == 0);
+      int sw_problem[2] = {-1, -1};  // problem of each switch not yet loaded
+      bool ok = true;
+      // Request the activations (and scales) of switch `j` into slot j & 1.
+      auto load_x = [&](int j) -> bool {
+        const int slot = j & 1;
+        if (j >= 2 && !mbar_wait(xempty_bar(slot), ((j >> 1) - 1) & 1, abort_flag)) return false;
+        const BatchProblem& P = bp.p[sw_problem[slot]];
+        xscal[4 * slot] =
+            *reinterpret_cast<const float*>(P.packed + static_cast<size_t>(P.n) * (P.k >> 2));
 #pragma unroll
-      for (int s = 0; s < S; ++s) {
-        issued_item[s] = -1;
-        issued_arrived[s] = false;
-      }
-      int it = 0;
-      for (int item = item_lo; item < item_hi && it < S; ++item, ++it) {
-        const int p = find_problem(bp, item);
-        const BatchProblem& P = bp.p[p];
-        const int row0 = (item - P.item_start) * P.rows_per_item;
-        const int nrows = min(P.rows_per_item, P.n - row0);
-        const uint32_t bytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(P.k >> 2);
-        mbar_expect_tx(full_bar(it), bytes);
-        bulk_load(smem_u32(stages + it * C::kStageBytes),
-                  P.packed + static_cast<size_t>(row0) * (P.k >> 2), bytes, full_bar(it));
-        issued_item[it] = it;
-      }
-      if (bp.pdl) grid_dependency_wait();
-      int prev_p = -1, nsw = 0;
-      it = 0;
-      for (int item = item_lo; item < item_hi; ++item, ++it) {
-        const int s = it % S;
-        const int p = find_problem(bp, item);
-        const BatchProblem& P = bp.p[p];
-        const int row0 = (item - P.item_start) * P.rows_per_item;
-        const int nrows = min(P.rows_per_item, P.n - row0);
-        if (it >= S) {
-          if (!mbar_wait(empty_bar(s), ((it / S) - 1) & 1, abort_flag)) break;
-          const uint32_t bytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(P.k >> 2);
-          mbar_expect_tx(full_bar(s), bytes);
-          bulk_load(smem_u32(stages + s * C::kStageBytes),
-                    P.packed + static_cast<size_t>(row0) * (P.k >> 2), bytes, full_bar(s));
-          issued_item[s] = it;
-          issued_arrived[s] = false;
+        for (int m = 0; m < MT; ++m) xscal[4 * slot + 1 + m] = (m < m_tokens) ? P.xs[m] : 0.0f;
+        const uint32_t xbytes = static_cast<uint32_t>(m_tokens) * static_cast<uint32_t>(P.k);
+        mbar_arrive_expect_tx(xfull_bar(slot), xbytes);  // publishes xscal[slot]
+        bulk_load(smem_u32(xslots + slot * C::kXSlotBytes), P.xq, xbytes, xfull_bar(slot));
+        return true;
+      };
+      auto load_pending_x = [&]() {
+        while (ok && x_loaded < nsw) {
+          ok = load_x(x_loaded);
+          ++x_loaded;
         }
-        int sw = -1;
-        if (p != prev_p) {
-          const int slot = nsw & 1;
-          if (nsw >= 2 && !mbar_wait(xempty_bar(slot), ((nsw >> 1) - 1) & 1, abort_flag)) break;
-          const uint32_t xbytes = static_cast<uint32_t>(m_tokens) * static_cast<uint32_t>(P.k);
-          // The scales, ahead of the consumers (published by the arrive below).
-          xscal[4 * slot] =
-              *reinterpret_cast<const float*>(P.packed + static_cast<size_t>(P.n) * (P.k >> 2));
-#pragma unroll
-          for (int m = 0; m < MT; ++m) xscal[4 * slot + 1 + m] = (m < m_tokens) ? P.xs[m] : 0.0f;
-          mbar_arrive_expect_tx(xfull_bar(slot), xbytes);
-          bulk_load(smem_u32(xslots + slot * C::kXSlotBytes), P.xq, xbytes, xfull_bar(slot));
-          sw = nsw++;
-          prev_p = p;
+      };
+      for (int item = item_lo; item < item_hi && ok; ++item) {
+        const int p = find_problem_by_item(bp, item);
+        const BatchProblem& P = bp.p[p];
+        const int row0 = (item - P.item_start) * kGemvTileRows;
+        const int nk = (P.k + 511) >> 9;
+        for (int kc = 0; kc < nk; ++kc) {
+          const int s = issued % S;
+          if (issued >= S) {
+            if (!waited) {
+              // Activations and scales come from the preceding grid.
+              grid_dependency_wait();
+              waited = true;
+              load_pending_x();
+              if (!ok) break;
+            }
+            if (!mbar_wait(empty_bar(s), ((issued / S) - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+          }
+          int info = (kc == 0 ? 1 : 0) | (kc == nk - 1 ? 2 : 0);
+          if (kc == 0 && p != prev_p) {
+            // At most two switches wait for their activations: the slots.
+            if (nsw - x_loaded >= 2) {
+              if (!waited) {
+                grid_dependency_wait();
+                waited = true;
+              }
+              load_pending_x();
+              if (!ok) break;
+            }
+            prefetch_tensormap(&bp.tmap[p]);
+            sw_problem[nsw & 1] = p;
+            info |= (nsw + 1) << 8;
+            ++nsw;
+            prev_p = p;
+          }
+          StageMeta md;
+          md.p = p;
+          md.row0 = row0;
+          md.kc = kc;
+          md.info = info;
+          meta[s] = md;
+          mbar_arrive_expect_tx(full_bar(s), C::kBoxBytes);  // publishes meta[s]
+          tma_load_2d(smem_u32(boxes + s * C::kBoxBytes), &bp.tmap[p], kc * 128, row0,
+                      full_bar(s));
+          ++issued;
+          if (waited) load_pending_x();
         }
-        StageMeta md;
-        md.p = p;
-        md.row0 = row0;
-        md.nrows = nrows;
-        md.sw = sw;
-        meta[s] = md;
-        mbar_arrive(full_bar(s));  // publishes meta[s]; the phase completes with the bytes
-        issued_arrived[s] = true;
       }
+      if (!waited) {
+        grid_dependency_wait();
+        waited = true;
+      }
+      load_pending_x();
       grid_dependents_launch();
       if (*abort_flag) {
-        // Let every copy still in flight land before shared memory goes away.
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-          if (issued_item[s] < 0) continue;
-          if (!issued_arrived[s]) mbar_arrive(full_bar(s));
-          mbar_wait(full_bar(s), (issued_item[s] / S) & 1, nullptr, kDrainTimeoutNs);
-        }
-        for (int j = 0; j < 2 && j < nsw; ++j) {
-          const int last = nsw - 1 - j;
-          mbar_wait(xfull_bar(last & 1), (last >> 1) & 1, nullptr, kDrainTimeoutNs);
-        }
+        // Let the copies still in flight land before shared memory goes away.
+        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+          mbar_wait(full_bar(i % S), (i / S) & 1, nullptr, kDrainTimeoutNs);
+        for (int j = (x_loaded > 2 ? x_loaded - 2 : 0); j < x_loaded; ++j)
+          mbar_wait(xfull_bar(j & 1), (j >> 1) & 1, nullptr, kDrainTimeoutNs);
       }
     }
     return;
@@ -229,116 +263,119 @@ __global__ void __launch_bounds__(GemvCfg<MT, WPL>::kThreads, 1)
 
   // ---------------------------------------------------------------- compute
   const int cw = warp - 1;
+  const int r = cw * 32 + lane;  // row of the tile owned by this lane
+  const int rsw = r & 7;         // its 128-byte swizzle phase
   if (bp.pdl) grid_dependency_wait();
-  uint32_t xr[MT][WPL][4];
+  int a[MT][4];
   int xsum[MT];
   float xsv[MT];
   float wscale = 0.0f;
-  int n = 0, k = 0, wr = 0;
-  float* yout = nullptr;
-  int32_t* accout = nullptr;
-  int it = 0;
-  for (int item = item_lo; item < item_hi; ++item, ++it) {
-    const int s = it % S;
-    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / S) & 1, abort_flag))) break;
+  const uint8_t* xsm = xslots;
+  int cur_slot = -1;
+  int k = 0, n = 0;
+  int nstages = 0;
+  for (int item = item_lo; item < item_hi; ++item)
+    nstages += (bp.p[find_problem_by_item(bp, item)].k + 511) >> 9;
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    xsum[m] = 0;
+    xsv[m] = 0.0f;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) a[m][g] = 0;
+  }
+  for (int i = 0; i < nstages; ++i) {
+    const int s = i % S;
+    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (i / S) & 1, abort_flag))) break;
     StageMeta md;
     {
       const volatile int32_t* vm = reinterpret_cast<const volatile int32_t*>(meta + s);
       md.p = vm[0];
       md.row0 = vm[1];
-      md.nrows = vm[2];
-      md.sw = vm[3];
+      md.kc = vm[2];
+      md.info = vm[3];
     }
-    if (md.sw >= 0) {
-      // A new problem: its activations into registers, then free the slot.
-      const int slot = md.sw & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(xfull_bar(slot), (md.sw >> 1) & 1, abort_flag)))
-        break;
-      const BatchProblem& P = bp.p[md.p];
-      n = P.n;
-      k = P.k;
-      wr = k >> 4;  // packed 32-bit words per row
-      yout = P.y;
-      accout = P.acc;
-      const uint8_t* xsm = xslots + slot * C::kXSlotBytes;
+    const int sw = (md.info >> 8) - 1;
+    if (sw >= 0) {
+      // A new problem: release the previous slot, take the new one.
+      if (cur_slot >= 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xempty_bar(cur_slot));
+      }
+      const int slot = sw & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(xfull_bar(slot), (sw >> 1) & 1, abort_flag))) break;
+      cur_slot = slot;
+      xsm = xslots + slot * C::kXSlotBytes;
+      k = bp.p[md.p].k;
+      n = bp.p[md.p].n;
+      wscale = xscal[4 * slot];
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
+        xsv[m] = xscal[4 * slot + 1 + m];
         int sum = 0;
-#pragma unroll
-        for (int t = 0; t < WPL; ++t) {
-          const int j = lane + 32 * t;
-          const bool live = (m < m_tokens) && (j < wr);
-          // word j of a row covers weights 128*(j/8) + 32*g + 4*(j%8) + {0..3}
-          const uint8_t* base = xsm + m * k + (j >> 3) * 128 + (j & 7) * 4;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const uint32_t v = live ? *reinterpret_cast<const uint32_t*>(base + 32 * g) : 0u;
-            xr[m][t][g] = v;
-            sum = __dp4a(static_cast<int>(v), 0x01010101, sum);
+        if (m < m_tokens) {
+          for (int off = lane * 16; off < k; off += 512) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xsm + m * k + off);
+            sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
+            sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
+            sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
+            sum = __dp4a(static_cast<int>(v.w), 0x01010101, sum);
           }
         }
         xsum[m] = __reduce_add_sync(0xffffffffu, sum);
       }
-      wscale = xscal[4 * slot];
-#pragma unroll
-      for (int m = 0; m < MT; ++m) xsv[m] = xscal[4 * slot + 1 + m];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xempty_bar(slot));
     }
-    const uint8_t* st = stages + s * C::kStageBytes;
-    const int rb = k >> 2;  // bytes per row
-    constexpr int R = C::kRowsPerPass;
-    for (int r0 = cw * R; r0 < md.nrows; r0 += C::kComputeWarps * R) {
-      const uint32_t* row[R];
-      bool has[R];
+    if (md.info & 1) {
 #pragma unroll
-      for (int q = 0; q < R; ++q) {
-        has[q] = r0 + q < md.nrows;
-        row[q] = reinterpret_cast<const uint32_t*>(st + static_cast<size_t>(has[q] ? r0 + q : r0) * rb);
-      }
-      int a[R][MT][4];
+      for (int m = 0; m < MT; ++m)
 #pragma unroll
-      for (int q = 0; q < R; ++q)
+        for (int g = 0; g < 4; ++g) a[m][g] = 0;
+    }
+    // One box: this lane's row in 8 chunks of 16 bytes (chunk c = words
+    // 4*(c&1)..+3 of I2_S block c>>1).  Blocks wholly past K are skipped.
+    const uint8_t* wrow = boxes + s * C::kBoxBytes + r * 128;
+    const int kbase = md.kc * 512;
+    const int nblk = min(4, (k - kbase) >> 7);
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
+    for (int c = 0; c < 8; ++c) {
+      if ((c >> 1) >= nblk) break;  // uniform over the warp
+      const uint4 w4 = *reinterpret_cast<const uint4*>(wrow + ((c ^ rsw) << 4));
+      const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      // group g of these words: k = kbase + 128*(c>>1) + 32*g + 16*(c&1) + 0..15
+      const uint8_t* xb = xsm + kbase + 128 * (c >> 1) + 16 * (c & 1);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) a[q][m][g] = 0;
+      for (int g = 0; g < 4; ++g) {
+        const uint32_t mask = 0x03030303u << (6 - 2 * g);
+        uint32_t v[4];
 #pragma unroll
-      for (int t = 0; t < WPL; ++t) {
-        if (32 * t >= wr) break;  // uniform over the warp
-        const int j = lane + 32 * t;
-        const bool live = j < wr;
-        uint32_t w[R];
-#pragma unroll
-        for (int q = 0; q < R; ++q) w[q] = (live && has[q]) ? row[q][j] : 0u;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t mask = 0x03030303u << (6 - 2 * g);
-#pragma unroll
-          for (int q = 0; q < R; ++q) {
-            const uint32_t v = w[q] & mask;
-#pragma unroll
-            for (int m = 0; m < MT; ++m) a[q][m][g] = dp4a_u8s8(v, xr[m][t][g], a[q][m][g]);
-          }
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < R; ++q) {
-        const int64_t nn = static_cast<int64_t>(md.row0) + r0 + q;
+        for (int q = 0; q < 4; ++q) v[q] = wv[q] & mask;
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          const int part = (a[q][m][0] >> 6) + (a[q][m][1] >> 4) + (a[q][m][2] >> 2) + a[q][m][3];
-          const int dot = __reduce_add_sync(0xffffffffu, part) - xsum[m];
-          if (has[q] && lane == m && m < m_tokens) {
-            yout[m * static_cast<int64_t>(n) + nn] =
-                __fmul_rn(__fmul_rn(__int2float_rn(dot), xsv[m]), wscale);
-            if (accout != nullptr) accout[m * static_cast<int64_t>(n) + nn] = dot;
-          }
+          const uint4 xv = *reinterpret_cast<const uint4*>(xb + m * k + 32 * g);
+          a[m][g] = dp4a_u8s8(v[0], xv.x, a[m][g]);
+          a[m][g] = dp4a_u8s8(v[1], xv.y, a[m][g]);
+          a[m][g] = dp4a_u8s8(v[2], xv.z, a[m][g]);
+          a[m][g] = dp4a_u8s8(v[3], xv.w, a[m][g]);
         }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));
+    if (md.info & 2) {
+      // Tile done: y = ((float)acc * xs[m]) * s for this lane's row.
+      const BatchProblem& P = bp.p[md.p];
+      const int64_t row = static_cast<int64_t>(md.row0) + r;
+      if (row < n) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          if (m < m_tokens) {
+            const int dot = (a[m][0] >> 6) + (a[m][1] >> 4) + (a[m][2] >> 2) + a[m][3] - xsum[m];
+            P.y[m * static_cast<int64_t>(n) + row] =
+                __fmul_rn(__fmul_rn(__int2float_rn(dot), xsv[m]), wscale);
+            if (P.acc != nullptr) P.acc[m * static_cast<int64_t>(n) + row] = dot;
+          }
+        }
+      }
+    }
   }
 }
 
