@@ -240,15 +240,18 @@ bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, int grid, cudaStream_t 
   return BITNET_OK;
 }
 
-// Persistent grid: two CTAs per SM, never more CTAs than row tiles.
+// Persistent grid: as many CTAs as fit on the SMs, never more than row tiles.
 template <int CAP>
 bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev) {
   bitnet_status st = plan_items(bp);
   if (st != BITNET_OK) return st;
   bp.pdl = pdl ? 1 : 0;
-  const int grid = std::min(bp.total_items, 2 * sm_count(dev));
-  return bp.m == 1 ? launch_dp4a_t<1, CAP>(bp, grid, stream, pdl, dev)
-                   : launch_dp4a_t<2, CAP>(bp, grid, stream, pdl, dev);
+  const int sms = sm_count(dev);
+  if (bp.m == 1)
+    return launch_dp4a_t<1, CAP>(bp, std::min(bp.total_items, GemvCfg<1>::kCtasPerSm * sms),
+                                 stream, pdl, dev);
+  return launch_dp4a_t<2, CAP>(bp, std::min(bp.total_items, GemvCfg<2>::kCtasPerSm * sms), stream,
+                               pdl, dev);
 }
 
 BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const float* x,

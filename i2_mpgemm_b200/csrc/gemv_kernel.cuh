@@ -15,12 +15,19 @@
 //     producer; on a change of problem it also copies the problem's int8
 //     activations (M x K bytes) into one of two x slots and stages the two
 //     scales next to them.
-//   * Warps 1..4 compute.  Lane l of warp w owns row 32w + l of the tile:
-//     it reads its row 16 bytes at a time (the swizzle makes the 8 lanes of
-//     each quarter-warp hit 8 different bank groups) and keeps int32
-//     accumulators for its row only, so no cross-lane reduction is needed
-//     and the tile's outputs are stored coalesced.  All lanes need the same
-//     activation bytes at the same time: those are 16-byte broadcast loads.
+//   * Warps 1..4 compute; warp w owns rows 32w..32w+31 of the tile.  Within
+//     a box, lane (rs, cp) = (lane / 4, lane % 4) owns I2_S block cp (32
+//     bytes, 128 weights) of the 4 rows 32w + rs + 8i, i = 0..3.  It loads
+//     the 128 activation bytes of its block into registers once per box and
+//     reuses them for its 4 rows, so shared-memory traffic is one read of
+//     each weight byte plus a quarter of an activation byte per weight byte
+//     (a broadcast read costs as many wavefronts as a plain one).  The
+//     128-byte swizzle makes the 8 lanes of each quarter-warp hit 8
+//     different bank groups for the weights; for the activations, lane cp
+//     visits the four groups starting at group cp, so the four blocks' reads
+//     of one instruction fall in four different 32-byte bank groups.  At the
+//     end of a tile the 4 lanes of a row add their partial sums with two
+//     shuffles.
 //
 // Unpack without shifts ("How BitNet's 1-Bit (I2_S) Quantization Works
 // Compared to Standard LLM Quantization", Ternary Representation and
@@ -79,7 +86,9 @@ struct GemvCfg {
   static constexpr int kComputeWarps = kGemvTileRows / 32;
   static constexpr int kThreads = 32 * (kComputeWarps + 1);
   static constexpr int kBoxBytes = kGemvTileRows * 128;  // 16 KB
-  static constexpr int kStages = 4;
+  // One token: 3 stages and 3 CTAs per SM; two tokens: 4 stages, 2 CTAs.
+  static constexpr int kStages = MT == 1 ? 3 : 4;
+  static constexpr int kCtasPerSm = MT == 1 ? 3 : 2;
   static constexpr int kXSlotBytes = MT * kGemvMaxK + 512;  // + slack read past K, never used
   static constexpr int kBars = 2 * kStages + 4;
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kBoxBytes +
@@ -123,7 +132,7 @@ __device__ __forceinline__ int first_item_at_stage(const BP& bp, int target) {
 }
 
 template <int MT, int CAP>
-__global__ void __launch_bounds__(GemvCfg<MT>::kThreads, 2)
+__global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm)
     i2s_gemv_dp4a_kernel(const __grid_constant__ BatchParamsT<CAP> bp) {
   using C = GemvCfg<MT>;
   constexpr int S = C::kStages;
@@ -263,10 +272,19 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, 2)
 
   // ---------------------------------------------------------------- compute
   const int cw = warp - 1;
-  const int r = cw * 32 + lane;  // row of the tile owned by this lane
-  const int rsw = r & 7;         // its 128-byte swizzle phase
+  const int rs = lane >> 2;  // row slot: rows 32*cw + rs + 8*i of the tile
+  const int cp = lane & 3;   // I2_S block of the box this lane reads
+  // Visit order of the groups for this lane: j -> group (j + cp) % 4.
+  uint32_t gmask[4];
+  int gshift[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int g = (j + cp) & 3;
+    gshift[j] = 6 - 2 * g;
+    gmask[j] = 0x03030303u << gshift[j];
+  }
   if (bp.pdl) grid_dependency_wait();
-  int a[MT][4];
+  int a[4][MT][4];  // [row i][token][visit j]: sum of code_g * x * 4^(3-g), g = (j + cp) % 4
   int xsum[MT];
   float xsv[MT];
   float wscale = 0.0f;
@@ -280,12 +298,16 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, 2)
   for (int m = 0; m < MT; ++m) {
     xsum[m] = 0;
     xsv[m] = 0.0f;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) a[m][g] = 0;
   }
-  for (int i = 0; i < nstages; ++i) {
-    const int s = i % S;
-    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (i / S) & 1, abort_flag))) break;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int g = 0; g < 4; ++g) a[i][m][g] = 0;
+  for (int it = 0; it < nstages; ++it) {
+    const int s = it % S;
+    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / S) & 1, abort_flag))) break;
     StageMeta md;
     {
       const volatile int32_t* vm = reinterpret_cast<const volatile int32_t*>(meta + s);
@@ -326,49 +348,70 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, 2)
     }
     if (md.info & 1) {
 #pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+          for (int g = 0; g < 4; ++g) a[i][m][g] = 0;
+    }
+    const int kblk = md.kc * 512 + 128 * cp;  // first weight of this lane's block
+    if (kblk < k) {                            // blocks wholly past K are skipped
+      // Activations of the block: group g, words 0..7 = k = kblk + 32g + 0..31,
+      // in this lane's visit order.
+      uint32_t xr[MT][4][8];
+#pragma unroll
       for (int m = 0; m < MT; ++m)
 #pragma unroll
-        for (int g = 0; g < 4; ++g) a[m][g] = 0;
-    }
-    // One box: this lane's row in 8 chunks of 16 bytes (chunk c = words
-    // 4*(c&1)..+3 of I2_S block c>>1).  Blocks wholly past K are skipped.
-    const uint8_t* wrow = boxes + s * C::kBoxBytes + r * 128;
-    const int kbase = md.kc * 512;
-    const int nblk = min(4, (k - kbase) >> 7);
+        for (int j = 0; j < 4; ++j) {
+          const uint8_t* xg = xsm + m * k + kblk + 32 * ((j + cp) & 3);
+          const uint4 lo = *reinterpret_cast<const uint4*>(xg);
+          const uint4 hi = *reinterpret_cast<const uint4*>(xg + 16);
+          xr[m][j][0] = lo.x;
+          xr[m][j][1] = lo.y;
+          xr[m][j][2] = lo.z;
+          xr[m][j][3] = lo.w;
+          xr[m][j][4] = hi.x;
+          xr[m][j][5] = hi.y;
+          xr[m][j][6] = hi.z;
+          xr[m][j][7] = hi.w;
+        }
+      const uint8_t* box = boxes + s * C::kBoxBytes;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      if ((c >> 1) >= nblk) break;  // uniform over the warp
-      const uint4 w4 = *reinterpret_cast<const uint4*>(wrow + ((c ^ rsw) << 4));
-      const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
-      // group g of these words: k = kbase + 128*(c>>1) + 32*g + 16*(c&1) + 0..15
-      const uint8_t* xb = xsm + kbase + 128 * (c >> 1) + 16 * (c & 1);
+      for (int i = 0; i < 4; ++i) {
+        const int r = cw * 32 + rs + 8 * i;  // row of the tile; r & 7 == rs
+        const uint8_t* wrow = box + r * 128;
+        const uint4 w0 = *reinterpret_cast<const uint4*>(wrow + (((2 * cp) ^ rs) << 4));
+        const uint4 w1 = *reinterpret_cast<const uint4*>(wrow + (((2 * cp + 1) ^ rs) << 4));
+        const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const uint32_t mask = 0x03030303u << (6 - 2 * g);
-        uint32_t v[4];
+        for (int j = 0; j < 4; ++j) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = wv[q] & mask;
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t v = wv[q] & gmask[j];
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(xb + m * k + 32 * g);
-          a[m][g] = dp4a_u8s8(v[0], xv.x, a[m][g]);
-          a[m][g] = dp4a_u8s8(v[1], xv.y, a[m][g]);
-          a[m][g] = dp4a_u8s8(v[2], xv.z, a[m][g]);
-          a[m][g] = dp4a_u8s8(v[3], xv.w, a[m][g]);
+            for (int m = 0; m < MT; ++m) a[i][m][j] = dp4a_u8s8(v, xr[m][j][q], a[i][m][j]);
+          }
         }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));
     if (md.info & 2) {
-      // Tile done: y = ((float)acc * xs[m]) * s for this lane's row.
+      // Tile done: add the 4 block lanes of each row, then
+      // y = ((float)acc * xs[m]) * s.
       const BatchProblem& P = bp.p[md.p];
-      const int64_t row = static_cast<int64_t>(md.row0) + r;
-      if (row < n) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t row = static_cast<int64_t>(md.row0) + cw * 32 + rs + 8 * i;
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          if (m < m_tokens) {
-            const int dot = (a[m][0] >> 6) + (a[m][1] >> 4) + (a[m][2] >> 2) + a[m][3] - xsum[m];
+          int part = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) part += a[i][m][j] >> gshift[j];
+          part += __shfl_xor_sync(0xffffffffu, part, 1);
+          part += __shfl_xor_sync(0xffffffffu, part, 2);
+          if (cp == 0 && m < m_tokens && row < n) {
+            const int dot = part - xsum[m];
             P.y[m * static_cast<int64_t>(n) + row] =
                 __fmul_rn(__fmul_rn(__int2float_rn(dot), xsv[m]), wscale);
             if (P.acc != nullptr) P.acc[m * static_cast<int64_t>(n) + row] = dot;
