@@ -554,6 +554,71 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
   return ok();
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of bitnet_i2s_quant_gemv.  Some callers have no way
+// to hand the library device scratch: a C plug-in that only receives raw
+// input and output pointers from a host framework that owns every allocation,
+// or a latency-critical loop that must never call the CUDA allocator (a
+// cudaMalloc can synchronize the device).  For them the scratch lives in a
+// fixed array in this library's device image, so every GPU that loads the
+// library holds it (1 MiB) until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t{1} << 20;
+
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device.  In host code the array's name is only a host-side stand-in, so
+// the address must come from the runtime; it is cached per device id.
+bitnet_status noalloc_scratch(int dev, void** out) {
+  static std::mutex mu;
+  static void* cached[kMaxDevices];
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
+    if (p == nullptr) return fail(BITNET_ERR_CUDA, "static scratch has no device address");
+    cached[dev] = p;
+  }
+  *out = cached[dev];
+  return BITNET_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bitnet_status bitnet_i2s_quant_gemv_noalloc(const uint8_t* packed, int64_t N, int64_t K,
+                                            const float* X, int64_t M, float* Y,
+                                            int32_t* acc_or_null, void* stream) {
+  const size_t need = bitnet_i2s_quant_gemv_workspace_bytes(M, K);
+  if (need != 0 && need > kNoAllocScratchBytes)
+    return fail(BITNET_ERR_SHAPE,
+                "bitnet_i2s_quant_gemv_noalloc: M=%lld x K=%lld needs %zu scratch bytes, more "
+                "than the %zu-byte static scratch (use bitnet_i2s_quant_gemv with a workspace)",
+                (long long)M, (long long)K, need, kNoAllocScratchBytes);
+  const float* dummy_xs = X;
+  bitnet_status st = check_matmul_args("bitnet_i2s_quant_gemv_noalloc", packed, N, K, X, dummy_xs,
+                                       M, Y, kMaxTokens);
+  if (st != BITNET_OK) return st;
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != BITNET_OK) return st;
+  // The quantizer writes every scratch byte the matmul then reads, so
+  // nothing left there by an earlier call is ever used.
+  return bitnet_i2s_quant_gemv(packed, N, K, X, M, Y, acc_or_null, scratch,
+                               kNoAllocScratchBytes, stream);
+}
+
 bitnet_status bitnet_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");

@@ -41,6 +41,7 @@ SIGNATURES = {
     "bitnet_i2s_quant_gemv_batched_workspace_bytes": (_SZ, [_VP, _I32, _I64]),
     "bitnet_i2s_quant_gemv_batched": (_I32, [_VP, _I32, _I64, _VP, _SZ, _VP]),
     "bitnet_i2s_gemv_batched": (_I32, [_VP, _I32, _I64, _VP]),
+    "bitnet_i2s_quant_gemv_noalloc": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP]),
     "bitnet_device_status": (_I32, []),
     "bitnet_last_error": (ctypes.c_char_p, []),
 }
@@ -261,6 +262,25 @@ class BatchedGemv:
 def bitnet_i2s_gemv_batched(problems, m: int, stream=None) -> None:
     """One call for many independent (packed, N, K, Xq, xs, Y, acc) problems."""
     BatchedGemv(problems, m).run(stream)
+
+
+def bitnet_i2s_quant_gemv_noalloc(packed, n, k, x, y=None, acc=None, want_acc=False,
+                                  stream=None):
+    """bitnet_i2s_quant_gemv using the library's static scratch (no workspace)."""
+    _need(packed, "packed", torch.uint8, bitnet_i2s_packed_bytes(n, k))
+    _need(x, "X", torch.float32)
+    m = x.shape[0]
+    _need(x, "X", torch.float32, m * k)
+    dev = packed.device
+    y = torch.empty((m, n), dtype=torch.float32, device=dev) if y is None else y
+    _need(y, "Y", torch.float32, m * n)
+    if want_acc and acc is None:
+        acc = torch.empty((m, n), dtype=torch.int32, device=dev)
+    if acc is not None:
+        _need(acc, "acc", torch.int32, m * n)
+    _check(lib.bitnet_i2s_quant_gemv_noalloc(_ptr(packed), n, k, _ptr(x), m, _ptr(y), _ptr(acc),
+                                             _stream(stream)))
+    return (y, acc) if acc is not None else y
 
 
 def bitnet_device_status() -> None:

@@ -184,6 +184,29 @@ typedef struct bitnet_i2s_qproblem {
 BITNET_API bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int count,
                                                  int64_t M, void* stream);
 
+/* bitnet_i2s_quant_gemv without a caller-supplied workspace, for callers
+ * that cannot allocate device memory: for example a plug-in that receives only
+ * raw input/output pointers from a host framework owning all allocations, or
+ * a latency-critical loop that must never enter the CUDA allocator.  (This
+ * entry point is a deployment convenience; the pages have no counterpart.)
+ *   - Scratch: a fixed 1 MiB array inside the library's device image, held by
+ *     every GPU that loads the library until the process exits.  The call
+ *     needs bitnet_i2s_quant_gemv_workspace_bytes(M,K) <= 1 MiB, i.e.
+ *     M*K rounded up to 256 plus 4*M rounded up to 256; larger shapes return
+ *     BITNET_ERR_SHAPE before anything is launched.
+ *   - It allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *     routine).  The first call on a device looks the array's address up
+ *     once for that device (with the device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array: two calls whose work may
+ *     overlap on the GPU (different streams, no ordering) race on it.  Calls
+ *     on one stream are ordered and safe.  Nothing in the array needs to
+ *     start at zero; each call overwrites what it reads.
+ *   Arguments and results as bitnet_i2s_quant_gemv. */
+BITNET_API bitnet_status bitnet_i2s_quant_gemv_noalloc(const uint8_t* packed, int64_t N, int64_t K,
+                                                       const float* X, int64_t M, float* Y,
+                                                       int32_t* acc_or_null, void* stream);
+
 /* Waits for all work on the current device, then returns
  * BITNET_ERR_DEVICE_TIMEOUT if any kernel of this library gave up on a
  * bounded wait since the last call (and clears the flag), BITNET_ERR_CUDA if
