@@ -43,6 +43,9 @@ METRIC = "I2_S ternary GEMV/GEMM: packed-weight GB/s & % HBM roofline; prefill T
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 NOMINAL_INT8_OVER_BF16 = 2.0  # 4.5 POPS int8 dense / 2.25 PFLOP/s bf16 dense
+DECODE_BATCH = 160  # problems per launch of the decode kernel
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "i2s_gemv_dp4a_stack_batch1.md")
+DECODE_SOURCE = os.path.join(ROOT, "i2_mpgemm_b200", "csrc", "gemv_kernel.cuh")
 
 
 # ------------------------------------------------------------------ setup
@@ -105,6 +108,28 @@ def load_peaks():
     except (OSError, KeyError, ValueError):
         return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
                 "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def measured_traffic():
+    """DRAM bytes per launch of the decode kernel from the committed ncu
+    summary, or None when the kernel's source changed since the capture."""
+    import hashlib
+    try:
+        text = open(TRAFFIC_SUMMARY).read()
+        src = hashlib.sha256(open(DECODE_SOURCE, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            key, _, val = line.strip()[2:].partition(":")
+            vals[key.strip()] = val.strip().strip("`")
+    if vals.get("kernel source sha256") != src:
+        return None
+    try:
+        return int(vals["dram bytes per launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 class ClockSampler:
@@ -263,7 +288,10 @@ def matmul_kernel_time(i2s, torch, probs, reps: int = 20):
     m = probs[0].m
     plan = i2s.BatchedGemv([(p.packed, p.n, p.k, q, s, p.y, None)
                             for p, (q, s) in zip(probs, qs)], m)
-    launches = 1 if (m <= 2 and max(p.k for p in probs) <= 8192) else len(probs)
+    # The decode kernel takes up to DECODE_BATCH problems per launch (M <= 2,
+    # K <= 8192); other problems run one launch each on the tensor-core kernel.
+    small = [p for p in probs if m <= 2 and p.k <= 8192]
+    launches = -(-len(small) // DECODE_BATCH) + (len(probs) - len(small))
     for _ in range(3):
         plan.run()
     torch.cuda.synchronize()
@@ -460,7 +488,7 @@ def run_native(args):
     achieved = k_bytes / (k_ms / 1000.0) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "peak_source": peaks["source"],
+                "traffic": measured_traffic(), "peak_source": peaks["source"],
                 "kernel": ("i2s_gemv_dp4a_kernel (one persistent launch over the 210 "
                            "projections)" if dp4a else "i2s_mma_kernel (one launch per projection)"),
                 "launches_per_step": k_launches,

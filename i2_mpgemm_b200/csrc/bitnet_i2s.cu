@@ -11,6 +11,8 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "bitnet_i2s.h"
 #include "gemv_kernel.cuh"
@@ -195,7 +197,7 @@ int sm_count(int dev) {
 // activations of one problem sit in a shared-memory slot); everything else
 // goes to the tensor-core kernel.
 constexpr int kMaxBatch = 160;  // problems per launch: the parameter block stays under 32 KB
-bool use_dp4a(int64_t m, int64_t kmax) { return m >= 1 && m <= 2 && kmax <= kGemvMaxK; }
+bool use_dp4a(int64_t m, int64_t k) { return m >= 1 && m <= 2 && k <= kGemvMaxK; }
 
 // Tensor maps, 128-row tiles and their stage counts for every problem.
 template <int CAP>
@@ -241,11 +243,15 @@ bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, int grid, cudaStream_t 
 }
 
 // Persistent grid: as many CTAs as fit on the SMs, never more than row tiles.
+// `pdl`: launch as a dependent of the preceding grid; `wait`: its CTAs wait
+// for that grid before reading activations (skipped only when the caller
+// knows the activations were complete before the preceding grid started).
 template <int CAP>
-bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev) {
+bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev,
+                          bool wait = true) {
   bitnet_status st = plan_items(bp);
   if (st != BITNET_OK) return st;
-  bp.pdl = pdl ? 1 : 0;
+  bp.pdl = (pdl && wait) ? 1 : 0;
   const int sms = sm_count(dev);
   if (bp.m == 1)
     return launch_dp4a_t<1, CAP>(bp, std::min(bp.total_items, GemvCfg<1>::kCtasPerSm * sms),
@@ -378,6 +384,58 @@ bitnet_status bitnet_i2s_gemm(const uint8_t* packed, int64_t N, int64_t K, const
   return st == BITNET_OK ? ok() : st;
 }
 
+bitnet_status bitnet_i2s_dequant_f32(const uint8_t* packed, int64_t N, int64_t K, float* W_out,
+                                     void* stream) {
+  if (packed == nullptr || W_out == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_dequant_f32: null pointer argument");
+  if (N < 1 || K < 128 || K % 128 != 0 || K > kMaxK)
+    return fail(BITNET_ERR_SHAPE, "bitnet_i2s_dequant_f32: N=%lld, K=%lld (K a multiple of 128)",
+                (long long)N, (long long)K);
+  if (!aligned(packed, 16) || !aligned(W_out, 16))
+    return fail(BITNET_ERR_ALIGN, "bitnet_i2s_dequant_f32: packed and W_out must be 16-byte aligned");
+  int dev;
+  bitnet_status st = check_device(&dev);
+  if (st != BITNET_OK) return st;
+  const int64_t words = N * K / 16;
+  const int grid = static_cast<int>(std::min<int64_t>((words + 255) / 256, int64_t{sm_count(dev)} * 16));
+  i2s_dequant_f32_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(packed), words,
+      reinterpret_cast<const float*>(packed + N * K / 4), W_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the dequantize kernel");
+  return ok();
+}
+
+size_t bitnet_ternarize_absmean_workspace_bytes(void) {
+  return static_cast<size_t>(kAbsMeanBlocks) * sizeof(double);
+}
+
+bitnet_status bitnet_ternarize_absmean(const float* W, int64_t count, double eps, float* W_out,
+                                       double* gamma_out, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  if (W == nullptr || W_out == nullptr || gamma_out == nullptr || workspace == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_ternarize_absmean: null pointer argument");
+  if (count < 1) return fail(BITNET_ERR_SHAPE, "bitnet_ternarize_absmean: count=%lld", (long long)count);
+  if (!(eps >= 0.0)) return fail(BITNET_ERR_INVALID_ARG, "bitnet_ternarize_absmean: eps must be >= 0");
+  if (workspace_bytes < bitnet_ternarize_absmean_workspace_bytes())
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_ternarize_absmean: workspace of %zu bytes < %zu",
+                workspace_bytes, bitnet_ternarize_absmean_workspace_bytes());
+  if (!aligned(W, 4) || !aligned(W_out, 4) || !aligned(gamma_out, 8) || !aligned(workspace, 8))
+    return fail(BITNET_ERR_ALIGN, "bitnet_ternarize_absmean: misaligned pointer");
+  int dev;
+  bitnet_status st = check_device(&dev);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* partial = static_cast<double*>(workspace);
+  absmean_partial_kernel<<<kAbsMeanBlocks, 256, 0, s>>>(W, count, partial);
+  absmean_finish_kernel<<<1, 32, 0, s>>>(partial, kAbsMeanBlocks, count, gamma_out);
+  const int grid = static_cast<int>(std::min<int64_t>((count + 255) / 256, int64_t{sm_count(dev)} * 16));
+  ternarize_kernel<<<grid, 256, 0, s>>>(W, count, eps, gamma_out, W_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the ternarization kernels");
+  return ok();
+}
+
 size_t bitnet_i2s_quant_gemv_workspace_bytes(int64_t M, int64_t K) {
   if (M < 1 || K < 128 || K % 128 != 0) return 0;
   return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
@@ -440,13 +498,11 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
     return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_quant_gemv_batched: no problems");
   if (M < 1 || M > kMaxTokens)
     return fail(BITNET_ERR_SHAPE, "bitnet_i2s_quant_gemv_batched: M=%lld", (long long)M);
-  int64_t kmax = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_i2s_problem& q = problems[i];
     bitnet_status st = check_matmul_args("bitnet_i2s_quant_gemv_batched", q.packed, q.N, q.K, q.X,
                                          q.X, M, q.Y, kMaxTokens);
     if (st != BITNET_OK) return st;
-    kmax = std::max(kmax, q.K);
   }
   if (workspace == nullptr)
     return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_quant_gemv_batched: null workspace");
@@ -463,52 +519,91 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
   if (st != BITNET_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const bool dp4a = use_dp4a(M, kmax);
-  static thread_local BatchParamsT<kMaxBatch> bp;  // 30 KB: kept off the stack
-  for (int base = 0; base < count; base += kMaxBatch) {
-    const int cnt = std::min(kMaxBatch, count - base);
-    bp.count = cnt;
-    bp.m = static_cast<int32_t>(M);
-    for (int i = 0; i < cnt; ++i) {
-      const bitnet_i2s_problem& q = problems[base + i];
-      int8_t* xq = reinterpret_cast<int8_t*>(ws);
-      float* xs = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(M) * q.K));
-      ws += bitnet_i2s_quant_gemv_workspace_bytes(M, q.K);
-      bp.p[i] = make_problem(q.packed, q.N, q.K, q.X, xq, xs, q.Y, q.acc_or_null);
+  // Problems the integer-ALU decode kernel serves: quantize all of them in
+  // one launch, then run the matmuls in launches of at most kMaxBatch
+  // problems (chunks of equal size).  The first matmul launch waits for the
+  // quantizer; the later ones are dependent launches that skip the wait and
+  // start streaming as soon as SMs free up: by the time they launch, every
+  // CTA of the first matmul launch has passed its own wait, so the
+  // quantizer has finished, and no matmul writes what another reads.
+  // The rest (K > 8192, or M > 2) run one by one on the tensor-core kernel.
+  static thread_local QuantBatchParams qp;              // 32 KB: kept off the stack
+  static thread_local BatchParamsT<kMaxBatch> bp;       // 30 KB
+  std::vector<int> small;
+  small.reserve(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    const bitnet_i2s_problem& q = problems[i];
+    int8_t* xq = reinterpret_cast<int8_t*>(ws);
+    float* xs = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(M) * q.K));
+    ws += bitnet_i2s_quant_gemv_workspace_bytes(M, q.K);
+    if (use_dp4a(M, q.K)) {
+      small.push_back(i);
+      continue;
     }
-    if (dp4a) {
-      // One launch quantizes every problem's tokens, one launch does every
-      // matmul; the second is a dependent launch of the first.
-      cudaLaunchConfig_t cfg;
-      std::memset(&cfg, 0, sizeof(cfg));
-      cfg.gridDim = dim3(static_cast<unsigned>(cnt * M));
-      cfg.blockDim = dim3(256);
-      cfg.stream = s;
-      cudaLaunchAttribute attr = pdl_attr(true);
-      cfg.attrs = &attr;
-      cfg.numAttrs = 1;
-      cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_batched_kernel<kMaxBatch>, bp);
-      if (e != cudaSuccess) return cuda_fail(e, "launch of the batched activation quant kernel");
-      st = launch_dp4a(bp, s, true, dev);
-      if (st != BITNET_OK) return st;
-    } else {
-      for (int i = 0; i < cnt; ++i) {
-        const BatchProblem& q = bp.p[i];
-        cudaLaunchConfig_t cfg;
-        std::memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3(static_cast<unsigned>(M));
-        cfg.blockDim = dim3(256);
-        cfg.stream = s;
-        cudaLaunchAttribute attr = pdl_attr(true);
-        cfg.attrs = &attr;
-        cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, q.x, static_cast<int64_t>(q.k),
-                                           q.xq, q.xs);
-        if (e != cudaSuccess) return cuda_fail(e, "launch of the activation quant kernel");
-        st = run_matmul(q.packed, q.n, q.k, q.xq, q.xs, M, q.y, q.acc, true, s, dev);
-        if (st != BITNET_OK) return st;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(M));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr = pdl_attr(true);
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, q.X, static_cast<int64_t>(q.K), xq, xs);
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the activation quant kernel");
+    st = run_matmul(q.packed, q.N, q.K, xq, xs, M, q.Y, q.acc_or_null, true, s, dev);
+    if (st != BITNET_OK) return st;
+  }
+  if (small.empty()) return ok();
+  // Workspace slices of the small problems, in call order.
+  std::vector<std::pair<int8_t*, float*>> sl(small.size());
+  {
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    size_t next = 0;
+    for (int i = 0; i < count && next < small.size(); ++i) {
+      if (small[next] == i) {
+        sl[next] = {reinterpret_cast<int8_t*>(w),
+                    reinterpret_cast<float*>(w + align256(static_cast<size_t>(M) * problems[i].K))};
+        ++next;
       }
+      w += bitnet_i2s_quant_gemv_workspace_bytes(M, problems[i].K);
     }
+  }
+  for (size_t base = 0; base < small.size(); base += kQuantBatch) {
+    const int cnt = static_cast<int>(std::min<size_t>(kQuantBatch, small.size() - base));
+    qp.count = cnt;
+    qp.m = static_cast<int32_t>(M);
+    for (int i = 0; i < cnt; ++i) {
+      const bitnet_i2s_problem& q = problems[small[base + i]];
+      qp.p[i].x = q.X;
+      qp.p[i].xq = sl[base + i].first;
+      qp.p[i].xs = sl[base + i].second;
+      qp.p[i].k = q.K;
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(cnt * M));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr = pdl_attr(true);
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_batched_kernel, qp);
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the batched activation quant kernel");
+  }
+  const int nchunks = static_cast<int>((small.size() + kMaxBatch - 1) / kMaxBatch);
+  const int per = static_cast<int>((small.size() + nchunks - 1) / nchunks);
+  for (int c = 0; c < nchunks; ++c) {
+    const size_t lo = static_cast<size_t>(c) * per;
+    const size_t hi = std::min(small.size(), lo + per);
+    bp.count = static_cast<int32_t>(hi - lo);
+    bp.m = static_cast<int32_t>(M);
+    for (size_t i = lo; i < hi; ++i) {
+      const bitnet_i2s_problem& q = problems[small[i]];
+      bp.p[i - lo] = make_problem(q.packed, q.N, q.K, q.X, sl[i].first, sl[i].second, q.Y,
+                                  q.acc_or_null);
+    }
+    st = launch_dp4a(bp, s, /*pdl=*/true, dev, /*wait=*/c == 0);
+    if (st != BITNET_OK) return st;
   }
   return ok();
 }
@@ -519,36 +614,45 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
     return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_gemv_batched: no problems");
   if (M < 1 || M > kMaxTokens)
     return fail(BITNET_ERR_SHAPE, "bitnet_i2s_gemv_batched: M=%lld", (long long)M);
-  int64_t kmax = 0;
   for (int i = 0; i < count; ++i) {
     const bitnet_i2s_qproblem& q = problems[i];
     bitnet_status st = check_matmul_args("bitnet_i2s_gemv_batched", q.packed, q.N, q.K, q.Xq,
                                          q.xs, M, q.Y, kMaxTokens);
     if (st != BITNET_OK) return st;
-    kmax = std::max(kmax, q.K);
   }
   int dev;
   bitnet_status st = check_device(&dev);
   if (st != BITNET_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (!use_dp4a(M, kmax)) {
-    for (int i = 0; i < count; ++i) {
-      const bitnet_i2s_qproblem& q = problems[i];
-      st = run_matmul(q.packed, q.N, q.K, q.Xq, q.xs, M, q.Y, q.acc_or_null, false, s, dev);
-      if (st != BITNET_OK) return st;
-    }
-    return ok();
-  }
+  // Problems the integer-ALU decode kernel serves run in launches of at most
+  // kMaxBatch problems (chunks of equal size).  The first launch is ordinary,
+  // so all earlier work on the stream has finished once it starts; the later
+  // ones are dependent launches that start as SMs free up.  The rest run one
+  // by one on the tensor-core kernel.
   static thread_local BatchParamsT<kMaxBatch> bp;
-  for (int base = 0; base < count; base += kMaxBatch) {
-    const int cnt = std::min(kMaxBatch, count - base);
-    bp.count = cnt;
-    bp.m = static_cast<int32_t>(M);
-    for (int i = 0; i < cnt; ++i) {
-      const bitnet_i2s_qproblem& q = problems[base + i];
-      bp.p[i] = make_problem(q.packed, q.N, q.K, nullptr, q.Xq, q.xs, q.Y, q.acc_or_null);
+  std::vector<int> small;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_i2s_qproblem& q = problems[i];
+    if (use_dp4a(M, q.K)) {
+      small.push_back(i);
+      continue;
     }
-    st = launch_dp4a(bp, s, false, dev);
+    st = run_matmul(q.packed, q.N, q.K, q.Xq, q.xs, M, q.Y, q.acc_or_null, false, s, dev);
+    if (st != BITNET_OK) return st;
+  }
+  if (small.empty()) return ok();
+  const int nchunks = static_cast<int>((small.size() + kMaxBatch - 1) / kMaxBatch);
+  const int per = static_cast<int>((small.size() + nchunks - 1) / nchunks);
+  for (int c = 0; c < nchunks; ++c) {
+    const size_t lo = static_cast<size_t>(c) * per;
+    const size_t hi = std::min(small.size(), lo + per);
+    bp.count = static_cast<int32_t>(hi - lo);
+    bp.m = static_cast<int32_t>(M);
+    for (size_t i = lo; i < hi; ++i) {
+      const bitnet_i2s_qproblem& q = problems[small[i]];
+      bp.p[i - lo] = make_problem(q.packed, q.N, q.K, nullptr, q.Xq, q.xs, q.Y, q.acc_or_null);
+    }
+    st = launch_dp4a(bp, s, /*pdl=*/c > 0, dev, /*wait=*/false);
     if (st != BITNET_OK) return st;
   }
   return ok();

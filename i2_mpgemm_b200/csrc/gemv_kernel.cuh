@@ -422,17 +422,31 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
   }
 }
 
-// Per-token absmax quantization of every problem's activations: one CTA per
-// (problem, token) row, the same arithmetic as act_quant_kernel.
-template <int CAP>
+// Per-token absmax quantization of many problems' activations in one launch:
+// one CTA per (problem, token) row, the same arithmetic as act_quant_kernel.
+constexpr int kQuantBatch = 1000;
+
+struct QuantProblem {
+  const float* x;  // [m, k] fp32
+  int8_t* xq;      // [m, k] int8
+  float* xs;       // [m]
+  int64_t k;
+};
+
+struct QuantBatchParams {
+  int32_t count;
+  int32_t m;
+  QuantProblem p[kQuantBatch];
+};
+
 __global__ void __launch_bounds__(256) act_quant_batched_kernel(
-    const __grid_constant__ BatchParamsT<CAP> bp) {
+    const __grid_constant__ QuantBatchParams qp) {
   grid_dependency_wait();
   grid_dependents_launch();
   __shared__ float red[32];
-  const int p = blockIdx.x / bp.m;
-  const int m = blockIdx.x % bp.m;
-  const BatchProblem& P = bp.p[p];
+  const int p = blockIdx.x / qp.m;
+  const int m = blockIdx.x % qp.m;
+  const QuantProblem& P = qp.p[p];
   quantize_row(P.x + static_cast<int64_t>(m) * P.k, P.k, P.xq + static_cast<int64_t>(m) * P.k,
                P.xs + m, red);
 }

@@ -124,4 +124,92 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict_
   quantize_row(x + row * k, k, xq + row * k, xs + row, red);
 }
 
+// ------------------------------------------------ dequantize to fp32 (to_float)
+// Full-tensor I2_S -> fp32: w_f32 = (code - 1) * s, exact ("ik_llama.cpp 运行
+// BitNet b1.58 2B 模型实战", section 5.1: an I2_S tensor is dequantized to f32 in
+// full before it is requantized).  One thread per packed 32-bit word writes
+// its 16 weights as four float4 (k = 32g + p .. p+3 of the block, g = 0..3).
+__global__ void __launch_bounds__(256) i2s_dequant_f32_kernel(const uint32_t* __restrict__ words,
+                                                              int64_t n_words,
+                                                              const float* __restrict__ scale,
+                                                              float* __restrict__ out) {
+  const float s = *scale;
+  for (int64_t wi = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; wi < n_words;
+       wi += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t w = __ldg(words + wi);
+    float* base = out + (wi >> 3) * kBlockWeights + static_cast<int>(wi & 7) * 4;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const int sh = 6 - 2 * g;
+      float4 v;
+      v.x = __fmul_rn(static_cast<float>(static_cast<int>((w >> sh) & 3u) - 1), s);
+      v.y = __fmul_rn(static_cast<float>(static_cast<int>((w >> (sh + 8)) & 3u) - 1), s);
+      v.z = __fmul_rn(static_cast<float>(static_cast<int>((w >> (sh + 16)) & 3u) - 1), s);
+      v.w = __fmul_rn(static_cast<float>(static_cast<int>((w >> (sh + 24)) & 3u) - 1), s);
+      *reinterpret_cast<float4*>(base + 32 * g) = v;
+    }
+  }
+}
+
+// ------------------------------------------------------ AbsMean ternarization
+// W~ = RoundClip(W / (gamma + eps), -1, 1), gamma = mean |W| ("LLM
+// Quantization Paradigms: FP8, AWQ, EXL2 & BitNet b1.58 in 2026", section 5,
+// The Mathematics of BitNet b1.58), the preprocessing step before packing.
+// gamma is a deterministic fp64 sum: every CTA adds its grid-stride share in
+// a fixed order into partial[blockIdx.x], then one CTA adds the partials in
+// index order.  The division and rounding are fp64 (ties away from zero);
+// the output is W~ * (float)gamma, which packs losslessly with scale gamma.
+constexpr int kAbsMeanBlocks = 1024;
+
+__device__ __forceinline__ double block_sum_f64(double v, double* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = (lane < static_cast<int>(blockDim.x >> 5)) ? red[lane] : 0.0;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+__global__ void __launch_bounds__(256) absmean_partial_kernel(const float* __restrict__ w,
+                                                              int64_t count,
+                                                              double* __restrict__ partial) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    acc += fabs(static_cast<double>(__ldg(w + i)));
+  acc = block_sum_f64(acc, red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = acc;
+}
+
+__global__ void __launch_bounds__(256) absmean_finish_kernel(const double* __restrict__ partial,
+                                                             int nparts, int64_t count,
+                                                             double* __restrict__ gamma_out) {
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < nparts; ++i) s += partial[i];
+    *gamma_out = s / static_cast<double>(count);
+  }
+}
+
+__global__ void __launch_bounds__(256) ternarize_kernel(const float* __restrict__ w, int64_t count,
+                                                        double eps, const double* __restrict__ gamma,
+                                                        float* __restrict__ out) {
+  const double g = *gamma;
+  const double den = g + eps;
+  const float gf = static_cast<float>(g);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const double t = static_cast<double>(__ldg(w + i)) / den;
+    const double r = fmin(1.0, fmax(-1.0, round(t)));
+    out[i] = static_cast<float>(r) * gf;
+  }
+}
+
 }  // namespace bitnet

@@ -36,6 +36,9 @@ SIGNATURES = {
     "bitnet_act_quant_i8": (_I32, [_VP, _I64, _I64, _VP, _VP, _VP]),
     "bitnet_i2s_gemv": (_I32, [_VP, _I64, _I64, _VP, _VP, _I64, _VP, _VP, _VP]),
     "bitnet_i2s_gemm": (_I32, [_VP, _I64, _I64, _VP, _VP, _I64, _VP, _VP, _VP]),
+    "bitnet_i2s_dequant_f32": (_I32, [_VP, _I64, _I64, _VP, _VP]),
+    "bitnet_ternarize_absmean_workspace_bytes": (_SZ, []),
+    "bitnet_ternarize_absmean": (_I32, [_VP, _I64, ctypes.c_double, _VP, _VP, _VP, _SZ, _VP]),
     "bitnet_i2s_quant_gemv_workspace_bytes": (_SZ, [_I64, _I64]),
     "bitnet_i2s_quant_gemv": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bitnet_i2s_quant_gemv_batched_workspace_bytes": (_SZ, [_VP, _I32, _I64]),
@@ -149,6 +152,28 @@ def bitnet_i2s_gemv(packed, n, k, xq, xs, y=None, acc=None, want_acc=False, stre
 def bitnet_i2s_gemm(packed, n, k, xq, xs, y=None, acc=None, want_acc=False, stream=None):
     """Matmul for any M >= 1: Y, or (Y, acc) with want_acc."""
     return _matmul(lib.bitnet_i2s_gemm, packed, n, k, xq, xs, y, acc, want_acc, stream)
+
+
+def bitnet_i2s_dequant_f32(packed, n, k, w_out=None, stream=None):
+    """I2_S tensor -> fp32 W[N,K] = (code - 1) * scale."""
+    _need(packed, "packed", torch.uint8, bitnet_i2s_packed_bytes(n, k))
+    w_out = torch.empty((n, k), dtype=torch.float32, device=packed.device) if w_out is None else w_out
+    _need(w_out, "W_out", torch.float32, n * k)
+    _check(lib.bitnet_i2s_dequant_f32(_ptr(packed), n, k, _ptr(w_out), _stream(stream)))
+    return w_out
+
+
+def bitnet_ternarize_absmean(w, eps: float = 1e-5, w_out=None, stream=None):
+    """AbsMean RoundClip ternarization: (W~ * gamma as fp32, gamma as a 1-element fp64 tensor)."""
+    _need(w, "W", torch.float32)
+    w_out = torch.empty_like(w) if w_out is None else w_out
+    _need(w_out, "W_out", torch.float32, w.numel())
+    gamma = torch.empty(1, dtype=torch.float64, device=w.device)
+    ws = torch.empty(int(lib.bitnet_ternarize_absmean_workspace_bytes()), dtype=torch.uint8,
+                     device=w.device)
+    _check(lib.bitnet_ternarize_absmean(_ptr(w), w.numel(), float(eps), _ptr(w_out), _ptr(gamma),
+                                        _ptr(ws), ws.numel(), _stream(stream)))
+    return w_out, gamma
 
 
 def bitnet_i2s_quant_gemv_workspace_bytes(m: int, k: int) -> int:

@@ -117,6 +117,32 @@ BITNET_API bitnet_status bitnet_i2s_gemm(const uint8_t* packed, int64_t N, int64
                               const float* xs, int64_t M, float* Y, int32_t* acc_or_null,
                               void* stream);
 
+/* Full-tensor dequantization I2_S -> fp32: W_out[n,k] = w[n,k] * s, exact
+ * ["ik_llama.cpp 运行 BitNet b1.58 2B 模型实战", section 5.1: an I2_S tensor is
+ * dequantized to f32 in full before being requantized; P1 "Ternary
+ * Representation and Packing" for the code layout].
+ * packed: I2_S tensor, 16-byte aligned.  W_out: N*K fp32, 16-byte aligned. */
+BITNET_API bitnet_status bitnet_i2s_dequant_f32(const uint8_t* packed, int64_t N, int64_t K,
+                                                float* W_out, void* stream);
+
+/* Device scratch bytes bitnet_ternarize_absmean needs (fixed, 8 KB). */
+BITNET_API size_t bitnet_ternarize_absmean_workspace_bytes(void);
+
+/* AbsMean ternarization, the preprocessing step before packing [P5 section
+ * 5, "The Mathematics of BitNet b1.58": W~ = RoundClip(W / (gamma + eps),
+ * -1, 1) with gamma = mean |W|; P2 Stage 1 applies it to the seven
+ * projections].
+ *   gamma is summed in fp64 in a fixed order (deterministic run to run) and
+ *   written to *gamma_out (device).  The division and the rounding (ties away
+ *   from zero) are fp64.  W_out[i] = W~[i] * (float)gamma, so
+ *   bitnet_i2s_pack(W_out) is lossless with scale (float)gamma.
+ *   W, W_out: `count` fp32 (may be the same buffer).  eps >= 0 (the pages
+ *   leave it open; 1e-5 is the usual choice).  workspace: at least
+ *   bitnet_ternarize_absmean_workspace_bytes(), 8-byte aligned. */
+BITNET_API bitnet_status bitnet_ternarize_absmean(const float* W, int64_t count, double eps,
+                                                  float* W_out, double* gamma_out, void* workspace,
+                                                  size_t workspace_bytes, void* stream);
+
 /* Bytes of device scratch that bitnet_i2s_quant_gemv needs for M tokens of
  * length K (the int8 activations and their scales).  0 for a bad shape. */
 BITNET_API size_t bitnet_i2s_quant_gemv_workspace_bytes(int64_t M, int64_t K);

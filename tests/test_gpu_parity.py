@@ -373,3 +373,45 @@ def test_gemv_batched_on_quantized_inputs(i2s, m):
         y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
         assert_acc_equal(pr[6].cpu().numpy(), acc_ref)
         assert_y_close(pr[5].cpu().numpy(), y_ref)
+
+
+# ------------------------------------------------ dequant and ternarization
+
+@pytest.mark.parametrize("n,k", [(1, 128), (7, 384), (130, 640), (640, 2560), (33, 6912)])
+def test_dequant_f32_is_exact(i2s, n, k):
+    w, t, s = inputs.ternary_weights(n, k, 8100 + n + k)
+    packed = oracle.pack(w.numpy())
+    got = i2s.bitnet_i2s_dequant_f32(dev(torch.from_numpy(packed)), n, k).cpu().numpy()
+    assert np.array_equal(got, oracle.dequant_f32(packed, n, k))
+    assert np.array_equal(got, w.numpy())  # lossless on ternary x scale
+
+
+@pytest.mark.parametrize("n,k", [(3, 128), (64, 2560), (640, 2560), (2560, 6912)])
+def test_ternarize_absmean_matches_oracle(i2s, n, k):
+    g = torch.Generator().manual_seed(n * 7 + k)
+    w = torch.randn((n, k), generator=g) * 0.02
+    out, gamma = i2s.bitnet_ternarize_absmean(dev(w), eps=1e-5)
+    out_ref, gamma_ref = oracle.ternarize_absmean(w.numpy(), eps=1e-5)
+    gam = float(gamma.cpu()[0])
+    # gamma: the same fp64 sum in another order, so equal up to rounding
+    assert abs(gam - gamma_ref) <= 1e-12 * abs(gamma_ref)
+    codes = np.sign(out.cpu().numpy())
+    codes_ref = np.sign(out_ref)
+    # the codes are decided in fp64 on both sides: identical unless |W/(gamma+eps)|
+    # lies within the gamma difference of 1/2, which these inputs never do
+    t = w.numpy().astype(np.float64) / (gamma_ref + 1e-5)
+    near_tie = np.abs(np.abs(t) - 0.5) < 1e-9
+    assert np.array_equal(codes[~near_tie], codes_ref[~near_tie])
+    assert np.array_equal(out.cpu().numpy(), codes.astype(np.float32) * np.float32(gam))
+    # the output packs losslessly with scale (float)gamma
+    t2, s2 = oracle.unpack(oracle.pack(out.cpu().numpy()), n, k)
+    if np.any(codes != 0):
+        assert s2 == np.float32(gam)
+    assert np.array_equal(t2, codes.astype(np.int8))
+
+
+def test_ternarize_worked_example_on_gpu(i2s):
+    w = torch.tensor([4, -4, 1, -1, 3, 0, 0, 3], dtype=torch.float32)
+    out, gamma = i2s.bitnet_ternarize_absmean(dev(w), eps=1e-5)
+    assert float(gamma.cpu()[0]) == 2.0
+    assert out.cpu().tolist() == [2.0, -2.0, 0.0, 0.0, 2.0, 0.0, 0.0, 2.0]
