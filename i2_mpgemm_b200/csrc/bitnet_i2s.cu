@@ -124,43 +124,6 @@ cudaLaunchAttribute pdl_attr(bool on) {
   return a;
 }
 
-template <int T, bool kCodes>
-bitnet_status launch_mma(const uint8_t* packed, int64_t n, int64_t k, const int8_t* xq,
-                         const float* xs, int64_t m, float* y, int32_t* acc, bool pdl,
-                         cudaStream_t stream, int dev) {
-  using C = MmaCfg<T, kCodes>;
-  static std::atomic<uint8_t> smem_done[kMaxDevices];
-  auto kern = i2s_mma_kernel<T, kCodes>;
-  bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
-  if (st != BITNET_OK) return st;
-  CUtensorMap tw, tx;
-  st = encode_u8_2d(&tw, packed, static_cast<uint64_t>(k / 4), static_cast<uint64_t>(n), 128, 128);
-  if (st != BITNET_OK) return st;
-  st = encode_u8_2d(&tx, xq, static_cast<uint64_t>(k), static_cast<uint64_t>(m), 128, T);
-  if (st != BITNET_OK) return st;
-  MmaParams p;
-  p.packed = packed;
-  p.xs = xs;
-  p.y = y;
-  p.acc = acc;
-  p.n = n;
-  p.k = k;
-  p.m = m;
-  p.pdl = pdl ? 1 : 0;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(static_cast<unsigned>((n + 127) / 128), static_cast<unsigned>((m + T - 1) / T));
-  cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr = pdl_attr(pdl);
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
-  if (e != cudaSuccess) return cuda_fail(e, "launch of the I2_S matmul kernel");
-  return BITNET_OK;
-}
-
 bitnet_status check_matmul_args(const char* fn, const uint8_t* packed, int64_t n, int64_t k,
                                 const void* x, const float* xs_or_dummy, int64_t m, float* y,
                                 int64_t max_m) {
@@ -276,8 +239,85 @@ BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const flo
   return q;
 }
 
-// Dispatch on the token count: small token tiles with the code-plus-correction
-// unpack for decode, 128-token tiles with the signed unpack for prefill.
+// ------------------------------------------------------ tensor-core path
+constexpr int kMmaBatch = 96;  // problems per launch: the parameter block stays under 32 KB
+
+// Tensor maps and item/chunk numbering for every problem of a batch.
+template <int T, int CAP>
+bitnet_status plan_mma(MmaParamsT<CAP>& bp, const int8_t* const* xq) {
+  const int64_t token_tiles = (bp.m + T - 1) / T;
+  int64_t items = 0, chunks = 0;
+  for (int i = 0; i < bp.count; ++i) {
+    MmaProblem& q = bp.p[i];
+    bitnet_status st = encode_u8_2d(&bp.tw[i], q.packed, static_cast<uint64_t>(q.k / 4),
+                                    static_cast<uint64_t>(q.n), 128, 128);
+    if (st != BITNET_OK) return st;
+    st = encode_u8_2d(&bp.tx[i], xq[i], static_cast<uint64_t>(q.k), static_cast<uint64_t>(bp.m),
+                      128, T);
+    if (st != BITNET_OK) return st;
+    q.item_start = static_cast<int32_t>(items);
+    q.chunk_start = static_cast<int32_t>(chunks);
+    const int64_t n_items = ((q.n + 127) / 128) * token_tiles;
+    items += n_items;
+    chunks += n_items * ((q.k + 511) / 512);
+    if (chunks > int64_t{0x7fffffff}) return fail(BITNET_ERR_SHAPE, "batch too large");
+  }
+  bp.total_items = static_cast<int32_t>(items);
+  bp.total_chunks = static_cast<int32_t>(chunks);
+  return BITNET_OK;
+}
+
+template <int T, bool kCodes, int CAP>
+bitnet_status launch_mma_t(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
+                           bool pdl, bool wait, int dev) {
+  using C = MmaCfg<T, kCodes>;
+  static std::atomic<uint8_t> smem_done[kMaxDevices];
+  auto kern = i2s_mma_kernel<T, kCodes, CAP>;
+  bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
+  if (st != BITNET_OK) return st;
+  if ((st = plan_mma<T>(bp, xq)) != BITNET_OK) return st;
+  bp.pdl = (pdl && wait) ? 1 : 0;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim =
+      dim3(static_cast<unsigned>(std::min(bp.total_items, C::kCtasPerSm * sm_count(dev))));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr = pdl_attr(pdl);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, bp);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the I2_S tensor-core kernel");
+  return BITNET_OK;
+}
+
+// Token tile by M: small tiles with unsigned codes for decode, 128-token
+// tiles with signed weights for prefill.
+template <int CAP>
+bitnet_status launch_mma(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
+                         bool pdl, bool wait, int dev) {
+  if (bp.m <= 16) return launch_mma_t<16, true>(bp, xq, stream, pdl, wait, dev);
+  if (bp.m <= 32) return launch_mma_t<32, true>(bp, xq, stream, pdl, wait, dev);
+  if (bp.m <= 64) return launch_mma_t<64, true>(bp, xq, stream, pdl, wait, dev);
+  return launch_mma_t<128, false>(bp, xq, stream, pdl, wait, dev);
+}
+
+MmaProblem make_mma_problem(const uint8_t* packed, int64_t n, int64_t k, const float* xs, float* y,
+                            int32_t* acc) {
+  MmaProblem q;
+  q.packed = packed;
+  q.xs = xs;
+  q.y = y;
+  q.acc = acc;
+  q.n = static_cast<int32_t>(n);
+  q.k = static_cast<int32_t>(k);
+  q.item_start = 0;
+  q.chunk_start = 0;
+  return q;
+}
+
+// One problem, on whichever kernel serves its shape.
 bitnet_status run_matmul(const uint8_t* packed, int64_t n, int64_t k, const int8_t* xq,
                          const float* xs, int64_t m, float* y, int32_t* acc, bool pdl,
                          cudaStream_t stream, int dev) {
@@ -288,10 +328,36 @@ bitnet_status run_matmul(const uint8_t* packed, int64_t n, int64_t k, const int8
     bp.p[0] = make_problem(packed, n, k, nullptr, xq, xs, y, acc);
     return launch_dp4a(bp, stream, pdl, dev);
   }
-  if (m <= 16) return launch_mma<16, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
-  if (m <= 32) return launch_mma<32, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
-  if (m <= 64) return launch_mma<64, true>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
-  return launch_mma<128, false>(packed, n, k, xq, xs, m, y, acc, pdl, stream, dev);
+  MmaParamsT<1> bp;
+  bp.count = 1;
+  bp.m = static_cast<int32_t>(m);
+  bp.p[0] = make_mma_problem(packed, n, k, xs, y, acc);
+  const int8_t* xqs[1] = {xq};
+  return launch_mma(bp, xqs, stream, pdl, true, dev);
+}
+
+// Many tensor-core problems sharing M: launches of at most kMmaBatch
+// problems in chunks of equal size, the first waiting for the preceding grid
+// (when `pdl`), the later ones dependent launches that skip the wait, as for
+// the decode batches.
+bitnet_status run_mma_batches(const std::vector<MmaProblem>& probs,
+                              const std::vector<const int8_t*>& xqs, int64_t m, bool pdl,
+                              cudaStream_t stream, int dev, bool wait_first = true) {
+  static thread_local MmaParamsT<kMmaBatch> bp;
+  const size_t total = probs.size();
+  if (total == 0) return BITNET_OK;
+  const size_t nchunks = (total + kMmaBatch - 1) / kMmaBatch;
+  for (size_t c = 0; c < nchunks; ++c) {
+    const size_t lo = total * c / nchunks;
+    const size_t hi = total * (c + 1) / nchunks;
+    bp.count = static_cast<int32_t>(hi - lo);
+    bp.m = static_cast<int32_t>(m);
+    for (size_t i = lo; i < hi; ++i) bp.p[i - lo] = probs[i];
+    bitnet_status st = launch_mma(bp, xqs.data() + lo, stream, c == 0 ? pdl : true,
+                                  c == 0 && wait_first, dev);
+    if (st != BITNET_OK) return st;
+  }
+  return BITNET_OK;
 }
 
 constexpr int64_t kMaxTokens = int64_t{65535} * 16;  // grid.y limit at the smallest tile
@@ -518,66 +584,35 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
   bitnet_status st = check_device(&dev);
   if (st != BITNET_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  // Problems the integer-ALU decode kernel serves: quantize all of them in
-  // one launch, then run the matmuls in launches of at most kMaxBatch
-  // problems (chunks of equal size).  The first matmul launch waits for the
-  // quantizer; the later ones are dependent launches that skip the wait and
-  // start streaming as soon as SMs free up: by the time they launch, every
-  // CTA of the first matmul launch has passed its own wait, so the
-  // quantizer has finished, and no matmul writes what another reads.
-  // The rest (K > 8192, or M > 2) run one by one on the tensor-core kernel.
-  static thread_local QuantBatchParams qp;              // 32 KB: kept off the stack
-  static thread_local BatchParamsT<kMaxBatch> bp;       // 30 KB
-  std::vector<int> small;
-  small.reserve(static_cast<size_t>(count));
-  for (int i = 0; i < count; ++i) {
-    const bitnet_i2s_problem& q = problems[i];
-    int8_t* xq = reinterpret_cast<int8_t*>(ws);
-    float* xs = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(M) * q.K));
-    ws += bitnet_i2s_quant_gemv_workspace_bytes(M, q.K);
-    if (use_dp4a(M, q.K)) {
-      small.push_back(i);
-      continue;
-    }
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(M));
-    cfg.blockDim = dim3(256);
-    cfg.stream = s;
-    cudaLaunchAttribute attr = pdl_attr(true);
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, q.X, static_cast<int64_t>(q.K), xq, xs);
-    if (e != cudaSuccess) return cuda_fail(e, "launch of the activation quant kernel");
-    st = run_matmul(q.packed, q.N, q.K, xq, xs, M, q.Y, q.acc_or_null, true, s, dev);
-    if (st != BITNET_OK) return st;
-  }
-  if (small.empty()) return ok();
-  // Workspace slices of the small problems, in call order.
-  std::vector<std::pair<int8_t*, float*>> sl(small.size());
+  // 1. One launch quantizes every problem's tokens into the workspace.
+  // 2. Problems the integer-ALU decode kernel serves (M <= 2, K <= 8192) run
+  //    in launches of at most kMaxBatch problems, the rest in launches of at
+  //    most kMmaBatch problems on the tensor-core kernel.
+  // The first matmul launch waits for the quantizer; every later one is a
+  // dependent launch that skips the wait and starts streaming as soon as SMs
+  // free up: each launch in the chain starts only after every CTA of the one
+  // before it has started, so all of them start after the quantizer has
+  // finished, and no matmul writes what another reads.
+  static thread_local QuantBatchParams qp;         // 32 KB: kept off the stack
+  static thread_local BatchParamsT<kMaxBatch> bp;  // 30 KB
+  std::vector<std::pair<int8_t*, float*>> sl(static_cast<size_t>(count));
   {
     uint8_t* w = static_cast<uint8_t*>(workspace);
-    size_t next = 0;
-    for (int i = 0; i < count && next < small.size(); ++i) {
-      if (small[next] == i) {
-        sl[next] = {reinterpret_cast<int8_t*>(w),
-                    reinterpret_cast<float*>(w + align256(static_cast<size_t>(M) * problems[i].K))};
-        ++next;
-      }
+    for (int i = 0; i < count; ++i) {
+      sl[i] = {reinterpret_cast<int8_t*>(w),
+               reinterpret_cast<float*>(w + align256(static_cast<size_t>(M) * problems[i].K))};
       w += bitnet_i2s_quant_gemv_workspace_bytes(M, problems[i].K);
     }
   }
-  for (size_t base = 0; base < small.size(); base += kQuantBatch) {
-    const int cnt = static_cast<int>(std::min<size_t>(kQuantBatch, small.size() - base));
+  for (int base = 0; base < count; base += kQuantBatch) {
+    const int cnt = std::min(kQuantBatch, count - base);
     qp.count = cnt;
     qp.m = static_cast<int32_t>(M);
     for (int i = 0; i < cnt; ++i) {
-      const bitnet_i2s_problem& q = problems[small[base + i]];
-      qp.p[i].x = q.X;
+      qp.p[i].x = problems[base + i].X;
       qp.p[i].xq = sl[base + i].first;
       qp.p[i].xs = sl[base + i].second;
-      qp.p[i].k = q.K;
+      qp.p[i].k = problems[base + i].K;
     }
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
@@ -590,19 +625,39 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
     cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_batched_kernel, qp);
     if (e != cudaSuccess) return cuda_fail(e, "launch of the batched activation quant kernel");
   }
-  const int nchunks = static_cast<int>((small.size() + kMaxBatch - 1) / kMaxBatch);
-  const int per = static_cast<int>((small.size() + nchunks - 1) / nchunks);
-  for (int c = 0; c < nchunks; ++c) {
-    const size_t lo = static_cast<size_t>(c) * per;
-    const size_t hi = std::min(small.size(), lo + per);
-    bp.count = static_cast<int32_t>(hi - lo);
-    bp.m = static_cast<int32_t>(M);
-    for (size_t i = lo; i < hi; ++i) {
-      const bitnet_i2s_problem& q = problems[small[i]];
-      bp.p[i - lo] = make_problem(q.packed, q.N, q.K, q.X, sl[i].first, sl[i].second, q.Y,
-                                  q.acc_or_null);
+  std::vector<int> small;
+  std::vector<MmaProblem> big;
+  std::vector<const int8_t*> big_xq;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_i2s_problem& q = problems[i];
+    if (use_dp4a(M, q.K)) {
+      small.push_back(i);
+    } else {
+      big.push_back(make_mma_problem(q.packed, q.N, q.K, sl[i].second, q.Y, q.acc_or_null));
+      big_xq.push_back(sl[i].first);
     }
-    st = launch_dp4a(bp, s, /*pdl=*/true, dev, /*wait=*/c == 0);
+  }
+  bool first = true;
+  if (!small.empty()) {
+    const size_t nchunks = (small.size() + kMaxBatch - 1) / kMaxBatch;
+    for (size_t c = 0; c < nchunks; ++c) {
+      const size_t lo = small.size() * c / nchunks;
+      const size_t hi = small.size() * (c + 1) / nchunks;
+      bp.count = static_cast<int32_t>(hi - lo);
+      bp.m = static_cast<int32_t>(M);
+      for (size_t i = lo; i < hi; ++i) {
+        const bitnet_i2s_problem& q = problems[small[i]];
+        bp.p[i - lo] = make_problem(q.packed, q.N, q.K, q.X, sl[small[i]].first,
+                                    sl[small[i]].second, q.Y, q.acc_or_null);
+      }
+      st = launch_dp4a(bp, s, /*pdl=*/true, dev, /*wait=*/first);
+      if (st != BITNET_OK) return st;
+      first = false;
+    }
+  }
+  if (!big.empty()) {
+    // run_mma_batches waits in its first launch only when asked to.
+    st = run_mma_batches(big, big_xq, M, /*pdl=*/true, s, dev, /*wait_first=*/first);
     if (st != BITNET_OK) return st;
   }
   return ok();
@@ -624,35 +679,42 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
   bitnet_status st = check_device(&dev);
   if (st != BITNET_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Problems the integer-ALU decode kernel serves run in launches of at most
-  // kMaxBatch problems (chunks of equal size).  The first launch is ordinary,
-  // so all earlier work on the stream has finished once it starts; the later
-  // ones are dependent launches that start as SMs free up.  The rest run one
-  // by one on the tensor-core kernel.
+  // Decode-kernel problems in launches of at most kMaxBatch, tensor-core
+  // problems in launches of at most kMmaBatch.  The first launch is
+  // ordinary, so all earlier work on the stream has finished once it
+  // starts; the later ones are dependent launches that start as SMs free up.
   static thread_local BatchParamsT<kMaxBatch> bp;
   std::vector<int> small;
+  std::vector<MmaProblem> big;
+  std::vector<const int8_t*> big_xq;
   for (int i = 0; i < count; ++i) {
     const bitnet_i2s_qproblem& q = problems[i];
     if (use_dp4a(M, q.K)) {
       small.push_back(i);
-      continue;
+    } else {
+      big.push_back(make_mma_problem(q.packed, q.N, q.K, q.xs, q.Y, q.acc_or_null));
+      big_xq.push_back(q.Xq);
     }
-    st = run_matmul(q.packed, q.N, q.K, q.Xq, q.xs, M, q.Y, q.acc_or_null, false, s, dev);
-    if (st != BITNET_OK) return st;
   }
-  if (small.empty()) return ok();
-  const int nchunks = static_cast<int>((small.size() + kMaxBatch - 1) / kMaxBatch);
-  const int per = static_cast<int>((small.size() + nchunks - 1) / nchunks);
-  for (int c = 0; c < nchunks; ++c) {
-    const size_t lo = static_cast<size_t>(c) * per;
-    const size_t hi = std::min(small.size(), lo + per);
-    bp.count = static_cast<int32_t>(hi - lo);
-    bp.m = static_cast<int32_t>(M);
-    for (size_t i = lo; i < hi; ++i) {
-      const bitnet_i2s_qproblem& q = problems[small[i]];
-      bp.p[i - lo] = make_problem(q.packed, q.N, q.K, nullptr, q.Xq, q.xs, q.Y, q.acc_or_null);
+  bool first = true;
+  if (!small.empty()) {
+    const size_t nchunks = (small.size() + kMaxBatch - 1) / kMaxBatch;
+    for (size_t c = 0; c < nchunks; ++c) {
+      const size_t lo = small.size() * c / nchunks;
+      const size_t hi = small.size() * (c + 1) / nchunks;
+      bp.count = static_cast<int32_t>(hi - lo);
+      bp.m = static_cast<int32_t>(M);
+      for (size_t i = lo; i < hi; ++i) {
+        const bitnet_i2s_qproblem& q = problems[small[i]];
+        bp.p[i - lo] = make_problem(q.packed, q.N, q.K, nullptr, q.Xq, q.xs, q.Y, q.acc_or_null);
+      }
+      st = launch_dp4a(bp, s, /*pdl=*/!first, dev, /*wait=*/false);
+      if (st != BITNET_OK) return st;
+      first = false;
     }
-    st = launch_dp4a(bp, s, /*pdl=*/c > 0, dev, /*wait=*/false);
+  }
+  if (!big.empty()) {
+    st = run_mma_batches(big, big_xq, M, /*pdl=*/!first, s, dev, /*wait_first=*/false);
     if (st != BITNET_OK) return st;
   }
   return ok();

@@ -415,3 +415,15 @@ def test_ternarize_worked_example_on_gpu(i2s):
     out, gamma = i2s.bitnet_ternarize_absmean(dev(w), eps=1e-5)
     assert float(gamma.cpu()[0]) == 2.0
     assert out.cpu().tolist() == [2.0, -2.0, 0.0, 0.0, 2.0, 0.0, 0.0, 2.0]
+
+
+def test_batched_tensor_path_over_several_launches(i2s):
+    # 4 tokens: every problem goes to the tensor-core kernel, 200 problems
+    # span several launches of the persistent kernel.
+    shapes = [(3 + 61 * (i % 4), 128 * (1 + i % 5)) for i in range(200)]
+    cases, problems = _batched_problems(shapes, 4, 6000)
+    i2s.bitnet_i2s_quant_gemv_batched(problems, 4)
+    for (packed, n, k, xq, xs), (_, _, _, _, y, acc) in zip(cases, problems):
+        y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+        assert_acc_equal(acc.cpu().numpy(), acc_ref, f"{n}x{k}")
+        assert_y_close(y.cpu().numpy(), y_ref, f"{n}x{k}")
