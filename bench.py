@@ -201,31 +201,56 @@ def gpu_uuid(torch, device_index: int) -> str | None:
 # ------------------------------------------------------------- workloads
 
 class Problem:
-    """One projection: resident packed weights plus its step buffers."""
+    """One projection: resident packed weights plus views of the step buffers."""
 
-    def __init__(self, i2s, torch, n, k, m, w, x_host):
+    def __init__(self, i2s, torch, n, k, m, w, x, y):
         self.n, self.k, self.m = n, k, m
         self.packed = i2s.bitnet_i2s_pack(w.cuda())
         self.packed_bytes = n * k // 4
-        self.x = x_host.cuda()
-        self.x_pinned = x_host.pin_memory()
-        self.y = torch.empty((m, n), dtype=torch.float32, device="cuda")
-        self.y_pinned = torch.empty((m, n), dtype=torch.float32).pin_memory()
+        self.x, self.y = x, y
         self.ws = torch.empty(i2s.bitnet_i2s_quant_gemv_workspace_bytes(m, k), dtype=torch.uint8,
                               device="cuda")
 
 
-def build_stack(i2s, torch, inputs, layers: int, m: int, act_seed_offset: int):
-    probs = []
-    for layer in range(layers):
-        for idx, p in enumerate(inputs.projections_2b()):
+class Stack:
+    """The projection stack with every input in one device buffer and every
+    output in another (each problem's X and Y are views), so an end-to-end
+    step moves its inputs and outputs with one copy each way."""
+
+    def __init__(self, i2s, torch, inputs, layers: int, m: int, act_seed_offset: int):
+        shapes = [(layer, idx, p) for layer in range(layers)
+                  for idx, p in enumerate(inputs.projections_2b())]
+        x_total = sum(m * p.k for _, _, p in shapes)
+        y_total = sum(m * p.n for _, _, p in shapes)
+        self.x_dev = torch.empty(x_total, dtype=torch.float32, device="cuda")
+        self.y_dev = torch.empty(y_total, dtype=torch.float32, device="cuda")
+        self.x_host = torch.empty(x_total, dtype=torch.float32).pin_memory()
+        self.y_host = torch.empty(y_total, dtype=torch.float32).pin_memory()
+        self.probs = []
+        xo = yo = 0
+        for layer, idx, p in shapes:
             seed = inputs.seed_stack(layer, idx)
             w, _, _ = inputs.ternary_weights(p.n, p.k, seed)
-            x = inputs.activations(m, p.k, seed + act_seed_offset)
-            probs.append(Problem(i2s, torch, p.n, p.k, m, w, x))
+            xv = inputs.activations(m, p.k, seed + act_seed_offset)
+            self.x_host[xo:xo + m * p.k].copy_(xv.reshape(-1))
+            x = self.x_dev[xo:xo + m * p.k].view(m, p.k)
+            y = self.y_dev[yo:yo + m * p.n].view(m, p.n)
+            self.probs.append(Problem(i2s, torch, p.n, p.k, m, w, x, y))
+            xo += m * p.k
+            yo += m * p.n
             del w
-    torch.cuda.synchronize()
-    return probs
+        self.x_dev.copy_(self.x_host)
+        torch.cuda.synchronize()
+
+    def h2d(self):
+        self.x_dev.copy_(self.x_host, non_blocking=True)
+
+    def d2h(self):
+        self.y_host.copy_(self.y_dev, non_blocking=True)
+
+
+def build_stack(i2s, torch, inputs, layers: int, m: int, act_seed_offset: int):
+    return Stack(i2s, torch, inputs, layers, m, act_seed_offset).probs
 
 
 def stack_step(i2s, probs):
@@ -428,7 +453,7 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1):
     # single k_proj GEMV (640 x 2560, batch 1): one launch vs graph steady state
     w, _, _ = inputs.ternary_weights(640, 2560, inputs.seed_single())
     x = inputs.activations(1, 2560, inputs.seed_single())
-    pr = Problem(i2s, torch, 640, 2560, 1, w, x)
+    pr = Problem(i2s, torch, 640, 2560, 1, w, x.cuda(), torch.empty((1, 640), device="cuda"))
     g = capture(torch, lambda: i2s.bitnet_i2s_quant_gemv(pr.packed, 640, 2560, pr.x, y=pr.y,
                                                          workspace=pr.ws))
     ms = time_replays(torch, g, 200, 10)
@@ -453,7 +478,8 @@ def run_native(args):
         raise SystemExit("--batch must be in 1..64")
 
     # Each rank: a replica of the weights, its own activations.
-    probs = build_stack(i2s, torch, inputs, args.layers, m, act_seed_offset=7919 * rank)
+    stack = Stack(i2s, torch, inputs, args.layers, m, act_seed_offset=7919 * rank)
+    probs = stack.probs
     packed_bytes = sum(p.packed_bytes for p in probs)
     plan = stack_batch(i2s, probs)
     dp4a = m <= 2
@@ -466,20 +492,12 @@ def run_native(args):
     clocks = clk.summary()
     value = world * packed_bytes / ms / 1e6  # GB/s over all ranks
 
-    # End to end through the public API: pinned inputs to the device, the
-    # step, the outputs back, every step.
-    h2d = sum(p.x.numel() * 4 for p in probs)
-    d2h = sum(p.y.numel() * 4 for p in probs)
-
-    def h2d_copy():
-        for p in probs:
-            p.x.copy_(p.x_pinned, non_blocking=True)
-
-    def d2h_copy():
-        for p in probs:
-            p.y_pinned.copy_(p.y, non_blocking=True)
-
-    ms_e2e = time_replays(torch, g, args.steps, args.warmup, before=h2d_copy, after=d2h_copy)
+    # End to end through the public API: every step copies all 210 inputs
+    # from pinned host memory to the device (one copy), runs the step and
+    # copies all outputs back (one copy).
+    h2d = stack.x_dev.numel() * 4
+    d2h = stack.y_dev.numel() * 4
+    ms_e2e = time_replays(torch, g, args.steps, args.warmup, before=stack.h2d, after=stack.d2h)
     ms_e2e = max_over_ranks(ms_e2e, dev)
     value_e2e = world * packed_bytes / ms_e2e / 1e6
 
@@ -489,8 +507,8 @@ def run_native(args):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": measured_traffic(), "peak_source": peaks["source"],
-                "kernel": ("i2s_gemv_dp4a_kernel (one persistent launch over the 210 "
-                           "projections)" if dp4a else "i2s_mma_kernel (one launch per projection)"),
+                "kernel": ("i2s_gemv_dp4a_kernel (persistent launches of up to 160 problems)"
+                           if dp4a else "i2s_mma_kernel (persistent launches of up to 96 problems)"),
                 "launches_per_step": k_launches,
                 "bytes_per_launch": int(k_bytes // k_launches),
                 "launch_us_mean": round(1000 * k_ms / k_launches, 3)}

@@ -785,6 +785,20 @@ bitnet_status bitnet_i2s_quant_gemv_noalloc(const uint8_t* packed, int64_t N, in
                                kNoAllocScratchBytes, stream);
 }
 
+bitnet_status bitnet_debug_wait_timeout(int64_t timeout_ns, void* stream) {
+  if (timeout_ns < 1000 || timeout_ns > 100000000)
+    return fail(BITNET_ERR_INVALID_ARG,
+                "bitnet_debug_wait_timeout: timeout_ns must be in [1e3, 1e8]");
+  int dev;
+  bitnet_status st = check_device(&dev);
+  if (st != BITNET_OK) return st;
+  stuck_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_ns));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the wait-timeout check");
+  return ok();
+}
+
 bitnet_status bitnet_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");

@@ -45,6 +45,7 @@ SIGNATURES = {
     "bitnet_i2s_quant_gemv_batched": (_I32, [_VP, _I32, _I64, _VP, _SZ, _VP]),
     "bitnet_i2s_gemv_batched": (_I32, [_VP, _I32, _I64, _VP]),
     "bitnet_i2s_quant_gemv_noalloc": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP]),
+    "bitnet_debug_wait_timeout": (_I32, [_I64, _VP]),
     "bitnet_device_status": (_I32, []),
     "bitnet_last_error": (ctypes.c_char_p, []),
 }
@@ -311,6 +312,11 @@ def bitnet_i2s_quant_gemv_noalloc(packed, n, k, x, y=None, acc=None, want_acc=Fa
 def bitnet_device_status() -> None:
     """Synchronize and raise BitnetError if a device-side wait ran out."""
     _check(lib.bitnet_device_status())
+
+
+def bitnet_debug_wait_timeout(timeout_ns: int = 1_000_000, stream=None) -> None:
+    """Launch one device wait that runs out after timeout_ns (failure-detection check)."""
+    _check(lib.bitnet_debug_wait_timeout(int(timeout_ns), _stream(stream)))
 
 
 def bitnet_last_error() -> str:

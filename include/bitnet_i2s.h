@@ -239,6 +239,14 @@ BITNET_API bitnet_status bitnet_i2s_quant_gemv_noalloc(const uint8_t* packed, in
  * the device reports an error, else BITNET_OK. */
 BITNET_API bitnet_status bitnet_device_status(void);
 
+/* Failure-detection check: launches one bounded device wait on a barrier
+ * that nothing completes, so it runs out after `timeout_ns` (1e3..1e8 ns)
+ * and raises the same device error flag a stuck pipeline would; the next
+ * bitnet_device_status() then returns BITNET_ERR_DEVICE_TIMEOUT and clears
+ * it.  Nothing faults or hangs: the kernel returns after the timeout.
+ * (A deployment check; the pages have no counterpart.) */
+BITNET_API bitnet_status bitnet_debug_wait_timeout(int64_t timeout_ns, void* stream);
+
 /* Message of the last error on this thread ("" if none). */
 BITNET_API const char* bitnet_last_error(void);
 

@@ -108,3 +108,8 @@ def test_product_package_never_touches_the_oracle():
                 text = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
                 assert "i2s_oracle" not in text, f
+
+
+def test_debug_wait_timeout_rejects_out_of_range_on_host(i2s):
+    assert i2s.lib.bitnet_debug_wait_timeout(10, None) == 1
+    assert i2s.lib.bitnet_debug_wait_timeout(10 ** 10, None) == 1

@@ -427,3 +427,17 @@ def test_batched_tensor_path_over_several_launches(i2s):
         y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
         assert_acc_equal(acc.cpu().numpy(), acc_ref, f"{n}x{k}")
         assert_y_close(y.cpu().numpy(), y_ref, f"{n}x{k}")
+
+
+# ------------------------------------------------------- failure detection
+
+def test_a_device_wait_that_runs_out_is_reported_and_cleared(i2s):
+    i2s.bitnet_device_status()  # start clean
+    i2s.bitnet_debug_wait_timeout(2_000_000)  # 2 ms, on a barrier nothing completes
+    with pytest.raises(i2s.BitnetError) as err:
+        i2s.bitnet_device_status()
+    assert err.value.status == 5  # BITNET_ERR_DEVICE_TIMEOUT
+    i2s.bitnet_device_status()  # the flag was cleared
+    # the context is still usable afterwards
+    w, _, _ = inputs.ternary_weights(7, 128, 3)
+    assert np.array_equal(i2s.bitnet_i2s_pack(dev(w)).cpu().numpy(), oracle.pack(w.numpy()))
