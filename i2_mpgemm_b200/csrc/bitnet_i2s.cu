@@ -590,9 +590,11 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
   //    most kMmaBatch problems on the tensor-core kernel.
   // The first matmul launch waits for the quantizer; every later one is a
   // dependent launch that skips the wait and starts streaming as soon as SMs
-  // free up: each launch in the chain starts only after every CTA of the one
-  // before it has started, so all of them start after the quantizer has
-  // finished, and no matmul writes what another reads.
+  // free up: each launch in the chain starts only after every thread of the
+  // one before it has signalled, which the first launch's threads do only
+  // after their wait, so all of them start after the quantizer has finished;
+  // no matmul writes what another reads; and every CTA waits for the grid
+  // before its own before it exits, so the last launch completes last.
   static thread_local QuantBatchParams qp;         // 32 KB: kept off the stack
   static thread_local BatchParamsT<kMaxBatch> bp;  // 30 KB
   std::vector<std::pair<int8_t*, float*>> sl(static_cast<size_t>(count));

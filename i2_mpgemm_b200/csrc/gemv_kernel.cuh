@@ -29,6 +29,13 @@
 //     end of a tile the 4 lanes of a row add their partial sums with two
 //     shuffles.
 //
+// Launch chaining (programmatic dependent launch): every thread signals the
+// next grid in the stream as soon as it has waited for its own inputs (at
+// once when the launch reads nothing the preceding grid writes), so the next
+// launch's CTAs take over SMs as soon as this launch's CTAs leave, and one
+// thread per CTA waits for the preceding grid before the CTA exits, so that
+// a grid never completes before the one it follows.
+//
 // Unpack without shifts ("How BitNet's 1-Bit (I2_S) Quantization Works
 // Compared to Standard LLM Quantization", Ternary Representation and
 // Packing: group g of a byte is bits [7-2g : 6-2g]): word & (3 << (6-2g)) in
@@ -175,12 +182,23 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane != 0) {
+      if (bp.pdl) grid_dependency_wait();
+      grid_dependents_launch();
+    } else {
       int issued = 0;    // boxes issued
       int nsw = 0;       // problem switches announced to the consumers
       int x_loaded = 0;  // switches whose activations were requested
       int prev_p = -1;
       bool waited = (bp.pdl == 0);
+      if (waited) grid_dependents_launch();
+      // The weights do not depend on the preceding grid: the first stages are
+      // issued before waiting for it.
+      auto wait_for_inputs = [&]() {
+        grid_dependency_wait();
+        grid_dependents_launch();
+        waited = true;
+      };
       int sw_problem[2] = {-1, -1};  // problem of each switch not yet loaded
       bool ok = true;
       // Request the activations (and scales) of switch `j` into slot j & 1.
@@ -213,8 +231,7 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
           if (issued >= S) {
             if (!waited) {
               // Activations and scales come from the preceding grid.
-              grid_dependency_wait();
-              waited = true;
+              wait_for_inputs();
               load_pending_x();
               if (!ok) break;
             }
@@ -227,10 +244,7 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
           if (kc == 0 && p != prev_p) {
             // At most two switches wait for their activations: the slots.
             if (nsw - x_loaded >= 2) {
-              if (!waited) {
-                grid_dependency_wait();
-                waited = true;
-              }
+              if (!waited) wait_for_inputs();
               load_pending_x();
               if (!ok) break;
             }
@@ -253,12 +267,11 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
           if (waited) load_pending_x();
         }
       }
-      if (!waited) {
-        grid_dependency_wait();
-        waited = true;
-      }
+      if (!waited) wait_for_inputs();
       load_pending_x();
-      grid_dependents_launch();
+      // This CTA does not finish before the preceding grid has, so that the
+      // completion of any grid in a chain implies that of all before it.
+      grid_dependency_wait();
       if (*abort_flag) {
         // Let the copies still in flight land before shared memory goes away.
         for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
@@ -284,6 +297,7 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
     gmask[j] = 0x03030303u << gshift[j];
   }
   if (bp.pdl) grid_dependency_wait();
+  grid_dependents_launch();
   int a[4][MT][4];  // [row i][token][visit j]: sum of code_g * x * 4^(3-g), g = (j + cp) % 4
   int xsum[MT];
   float xsv[MT];

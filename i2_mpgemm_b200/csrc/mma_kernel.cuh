@@ -209,6 +209,17 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
   const int item_lo = mma_first_item_at(bp, static_cast<int>(tc * blockIdx.x / gridDim.x));
   const int item_hi = mma_first_item_at(bp, static_cast<int>(tc * (blockIdx.x + 1) / gridDim.x));
 
+  // Launch chaining: every thread but the producer signals the next grid
+  // once it has waited for this grid's inputs (at once when the launch reads
+  // nothing the preceding grid writes); the producer does so after its own
+  // lazy wait, and waits once more for the preceding grid before it exits.
+  // The stages every role consumes carry activations, which the producer
+  // requests only after its wait, so the other roles lose nothing by waiting.
+  if (warp != 0 || lane != 0) {
+    if (bp.pdl) grid_dependency_wait();
+    grid_dependents_launch();
+  }
+
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -217,6 +228,7 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
       // the weight and activation bytes together.
       int issued = 0;
       bool waited = (bp.pdl == 0);
+      if (waited) grid_dependents_launch();
       bool ok = true;
       int pre_item = item_lo, pre_kc = 0;  // chunk cursor of the activation loads
       auto chunk_blocks = [&](const MmaProblem& P, int kc) { return min(4, (P.k >> 7) - 4 * kc); };
@@ -242,6 +254,7 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
           if (issued >= S) {
             if (!waited) {
               grid_dependency_wait();
+              grid_dependents_launch();
               waited = true;
               for (int i = 0; i < S; ++i) {  // activations of the stages issued so far
                 issue_x(i, pre_item, pre_kc);
@@ -268,6 +281,7 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
       }
       if (!waited && ok) {
         grid_dependency_wait();
+        grid_dependents_launch();
         waited = true;
         for (int i = 0; i < issued; ++i) {
           issue_x(i, pre_item, pre_kc);
@@ -279,7 +293,9 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
           }
         }
       }
-      grid_dependents_launch();
+      // This CTA does not finish before the preceding grid has, so that the
+      // completion of any grid in a chain implies that of all before it.
+      grid_dependency_wait();
       if (*abort_flag) {
         // Let the copies already issued land before shared memory goes away
         // (a stage whose activations were never requested cannot complete;
@@ -431,7 +447,6 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    if (bp.pdl) grid_dependency_wait();
     int ii = 0;
     for (int item = item_lo; item < item_hi; ++item, ++ii) {
       int p, rt, tt;
