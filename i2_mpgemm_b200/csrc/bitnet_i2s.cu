@@ -160,11 +160,20 @@ int sm_count(int dev) {
 // activations of one problem sit in a shared-memory slot); everything else
 // goes to the tensor-core kernel.
 constexpr int kMaxBatch = 160;  // problems per launch: the parameter block stays under 32 KB
+// With a work queue, the share of a decode launch's stages in fixed per-CTA
+// ranges; the rest is handed out at run time.
+constexpr double kStaticShare = 0.7;
 bool use_dp4a(int64_t m, int64_t k) { return m >= 1 && m <= 2 && k <= kGemvMaxK; }
 
 // Tensor maps, 128-row tiles and their stage counts for every problem.
 template <int CAP>
 bitnet_status plan_items(BatchParamsT<CAP>& bp) {
+  if (bp.queue != nullptr) {
+    // Items are handed out in order: the longest ones (largest K) first, so
+    // that the last items taken are short and the CTAs end together.
+    std::stable_sort(bp.p, bp.p + bp.count,
+                     [](const BatchProblem& a, const BatchProblem& b) { return a.k > b.k; });
+  }
   int64_t items = 0, stages = 0;
   for (int i = 0; i < bp.count; ++i) {
     BatchProblem& q = bp.p[i];
@@ -180,6 +189,24 @@ bitnet_status plan_items(BatchParamsT<CAP>& bp) {
   }
   bp.total_items = static_cast<int32_t>(items);
   bp.total_stages = static_cast<int32_t>(stages);
+  // Without a queue every item sits in a fixed range; with one, the items
+  // after the first kStaticShare of the stages are handed out at run time.
+  bp.dyn_start = bp.total_items;
+  bp.static_stages = bp.total_stages;
+  if (bp.queue != nullptr) {
+    const int64_t cut = static_cast<int64_t>(kStaticShare * static_cast<double>(stages));
+    for (int i = 0; i < bp.count; ++i) {
+      const BatchProblem& q = bp.p[i];
+      const int64_t nk = (q.k + 511) / 512;
+      const int64_t tiles = (q.n + kGemvTileRows - 1) / kGemvTileRows;
+      if (q.stage_start + tiles * nk > cut) {
+        const int64_t off = std::max<int64_t>(0, (cut - q.stage_start + nk - 1) / nk);
+        bp.dyn_start = static_cast<int32_t>(q.item_start + std::min(off, tiles));
+        bp.static_stages = static_cast<int32_t>(q.stage_start + std::min(off, tiles) * nk);
+        break;
+      }
+    }
+  }
   return BITNET_OK;
 }
 
@@ -325,6 +352,7 @@ bitnet_status run_matmul(const uint8_t* packed, int64_t n, int64_t k, const int8
     BatchParamsT<1> bp;
     bp.count = 1;
     bp.m = static_cast<int32_t>(m);
+    bp.queue = nullptr;
     bp.p[0] = make_problem(packed, n, k, nullptr, xq, xs, y, acc);
     return launch_dp4a(bp, stream, pdl, dev);
   }
@@ -363,6 +391,11 @@ bitnet_status run_mma_batches(const std::vector<MmaProblem>& probs,
 constexpr int64_t kMaxTokens = int64_t{65535} * 16;  // grid.y limit at the smallest tile
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// Work counters of the decode launches of a batch of `count` problems.
+size_t queue_bytes(int count) {
+  return align256(sizeof(int32_t) * static_cast<size_t>((count + kMaxBatch - 1) / kMaxBatch));
+}
 
 }  // namespace
 
@@ -554,7 +587,7 @@ size_t bitnet_i2s_quant_gemv_batched_workspace_bytes(const bitnet_i2s_problem* p
     if (one == 0) return 0;
     total += one;
   }
-  return total;
+  return total + queue_bytes(count);
 }
 
 bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, int count,
@@ -598,6 +631,7 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
   static thread_local QuantBatchParams qp;         // 32 KB: kept off the stack
   static thread_local BatchParamsT<kMaxBatch> bp;  // 30 KB
   std::vector<std::pair<int8_t*, float*>> sl(static_cast<size_t>(count));
+  int32_t* queue = nullptr;  // the decode launches' work counters, after the slots
   {
     uint8_t* w = static_cast<uint8_t*>(workspace);
     for (int i = 0; i < count; ++i) {
@@ -605,11 +639,16 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
                reinterpret_cast<float*>(w + align256(static_cast<size_t>(M) * problems[i].K))};
       w += bitnet_i2s_quant_gemv_workspace_bytes(M, problems[i].K);
     }
+    queue = reinterpret_cast<int32_t*>(w);
   }
   for (int base = 0; base < count; base += kQuantBatch) {
     const int cnt = std::min(kQuantBatch, count - base);
     qp.count = cnt;
     qp.m = static_cast<int32_t>(M);
+    // The first quantizer launch zeroes the counters; every decode launch
+    // reads its counter only once the quantizers have finished.
+    qp.queue = base == 0 ? queue : nullptr;
+    qp.nqueue = base == 0 ? static_cast<int32_t>(queue_bytes(count) / sizeof(int32_t)) : 0;
     for (int i = 0; i < cnt; ++i) {
       qp.p[i].x = problems[base + i].X;
       qp.p[i].xq = sl[base + i].first;
@@ -647,6 +686,7 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
       const size_t hi = small.size() * (c + 1) / nchunks;
       bp.count = static_cast<int32_t>(hi - lo);
       bp.m = static_cast<int32_t>(M);
+      bp.queue = queue + c;
       for (size_t i = lo; i < hi; ++i) {
         const bitnet_i2s_problem& q = problems[small[i]];
         bp.p[i - lo] = make_problem(q.packed, q.N, q.K, q.X, sl[small[i]].first,
@@ -665,8 +705,12 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
   return ok();
 }
 
+size_t bitnet_i2s_gemv_batched_workspace_bytes(int count) {
+  return count < 1 ? 0 : queue_bytes(count);
+}
+
 bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int count, int64_t M,
-                                      void* stream) {
+                                      void* workspace, size_t workspace_bytes, void* stream) {
   if (problems == nullptr || count < 1)
     return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_gemv_batched: no problems");
   if (M < 1 || M > kMaxTokens)
@@ -677,10 +721,22 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
                                          q.xs, M, q.Y, kMaxTokens);
     if (st != BITNET_OK) return st;
   }
+  if (workspace != nullptr) {
+    if (!aligned(workspace, 256))
+      return fail(BITNET_ERR_ALIGN, "bitnet_i2s_gemv_batched: workspace must be 256-byte aligned");
+    if (workspace_bytes < queue_bytes(count))
+      return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_gemv_batched: workspace of %zu bytes < %zu",
+                  workspace_bytes, queue_bytes(count));
+  }
   int dev;
   bitnet_status st = check_device(&dev);
   if (st != BITNET_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* queue = static_cast<int32_t*>(workspace);
+  if (queue != nullptr) {
+    cudaError_t e = cudaMemsetAsync(queue, 0, queue_bytes(count), s);
+    if (e != cudaSuccess) return cuda_fail(e, "zeroing the work counters");
+  }
   // Decode-kernel problems in launches of at most kMaxBatch, tensor-core
   // problems in launches of at most kMmaBatch.  The first launch is
   // ordinary, so all earlier work on the stream has finished once it
@@ -706,6 +762,7 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
       const size_t hi = small.size() * (c + 1) / nchunks;
       bp.count = static_cast<int32_t>(hi - lo);
       bp.m = static_cast<int32_t>(M);
+      bp.queue = queue != nullptr ? queue + c : nullptr;
       for (size_t i = lo; i < hi; ++i) {
         const bitnet_i2s_qproblem& q = problems[small[i]];
         bp.p[i - lo] = make_problem(q.packed, q.N, q.K, nullptr, q.Xq, q.xs, q.Y, q.acc_or_null);

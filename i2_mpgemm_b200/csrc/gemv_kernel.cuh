@@ -75,7 +75,10 @@ struct BatchParamsT {
   int32_t total_items;   // row tiles over all problems
   int32_t total_stages;  // boxes over all problems
   int32_t pdl;           // 1: activations come from the preceding grid
-  int32_t pad[11];
+  int32_t dyn_start;     // items from here on are handed out through `queue`
+  int32_t* queue;        // zeroed work counter, or null: every item in a fixed range
+  int32_t static_stages; // stages of the items before dyn_start
+  int32_t pad[7];
   CUtensorMap tmap[CAP];  // per problem: packed bytes as [n rows, k/4 bytes], box 128 x 128
   BatchProblem p[CAP];
 };
@@ -176,7 +179,8 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
   __syncthreads();
 
   const int m_tokens = bp.m;
-  const int64_t ts = bp.total_stages;
+  // Fixed ranges over the items before dyn_start, balanced by stages.
+  const int64_t ts = bp.static_stages;
   const int item_lo = first_item_at_stage(bp, static_cast<int>(ts * blockIdx.x / gridDim.x));
   const int item_hi = first_item_at_stage(bp, static_cast<int>(ts * (blockIdx.x + 1) / gridDim.x));
 
@@ -192,6 +196,18 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
       int prev_p = -1;
       bool waited = (bp.pdl == 0);
       if (waited) grid_dependents_launch();
+      // Items: first this CTA's fixed range, then, with a work queue, items
+      // from dyn_start on, one at a time, as the CTA becomes free (the counter
+      // is zeroed by the preceding grid, so it is read only after the wait).
+      // The fixed ranges keep every CTA on neighbouring tiles of one problem
+      // for most of the launch; the shared tail evens out the finishing times.
+      const bool dyn = bp.queue != nullptr;
+      int next = 0;
+      bool have_next = false;
+      auto grab = [&]() {  // its result is used one item later
+        next = bp.dyn_start + atomicAdd(bp.queue, 1);
+        have_next = true;
+      };
       // The weights do not depend on the preceding grid: the first stages are
       // issued before waiting for it.
       auto wait_for_inputs = [&]() {
@@ -199,6 +215,9 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
         grid_dependents_launch();
         waited = true;
       };
+      // Weights are read once: they go first when L2 needs room, so that the
+      // activations the next CTAs read stay there.
+      const uint64_t pol_w = l2_policy_evict_first();
       int sw_problem[2] = {-1, -1};  // problem of each switch not yet loaded
       bool ok = true;
       // Request the activations (and scales) of switch `j` into slot j & 1.
@@ -221,7 +240,22 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
           ++x_loaded;
         }
       };
-      for (int item = item_lo; item < item_hi && ok; ++item) {
+      int item = item_lo;
+      bool in_static = item_lo < item_hi;
+      if (!in_static) {
+        if (dyn) {
+          if (!waited) wait_for_inputs();
+          grab();
+          item = next;
+          have_next = false;
+        } else {
+          item = bp.total_items;
+        }
+      }
+      while (ok && item < bp.total_items) {
+        // The next shared item is requested while the last fixed one (or a
+        // shared one) is issued, so the atomic's round trip is hidden.
+        if (dyn && waited && !have_next && (!in_static || item + 1 >= item_hi)) grab();
         const int p = find_problem_by_item(bp, item);
         const BatchProblem& P = bp.p[p];
         const int row0 = (item - P.item_start) * kGemvTileRows;
@@ -261,14 +295,41 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
           md.info = info;
           meta[s] = md;
           mbar_arrive_expect_tx(full_bar(s), C::kBoxBytes);  // publishes meta[s]
-          tma_load_2d(smem_u32(boxes + s * C::kBoxBytes), &bp.tmap[p], kc * 128, row0,
-                      full_bar(s));
+          tma_load_2d_hint(smem_u32(boxes + s * C::kBoxBytes), &bp.tmap[p], kc * 128, row0,
+                           full_bar(s), pol_w);
           ++issued;
           if (waited) load_pending_x();
+        }
+        if (!ok) break;
+        if (in_static && item + 1 < item_hi) {
+          ++item;
+        } else if (dyn) {
+          if (!have_next) {
+            if (!waited) wait_for_inputs();
+            grab();
+          }
+          item = next;
+          have_next = false;
+          in_static = false;
+        } else {
+          break;
         }
       }
       if (!waited) wait_for_inputs();
       load_pending_x();
+      if (ok) {
+        // End of the work: a stage without data whose meta says so.
+        const int s = issued % S;
+        if (issued < S || mbar_wait(empty_bar(s), ((issued / S) - 1) & 1, abort_flag)) {
+          StageMeta md;
+          md.p = -1;
+          md.row0 = 0;
+          md.kc = 0;
+          md.info = 0;
+          meta[s] = md;
+          mbar_arrive(full_bar(s));  // publishes meta[s]
+        }
+      }
       // This CTA does not finish before the preceding grid has, so that the
       // completion of any grid in a chain implies that of all before it.
       grid_dependency_wait();
@@ -305,9 +366,6 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
   const uint8_t* xsm = xslots;
   int cur_slot = -1;
   int k = 0, n = 0;
-  int nstages = 0;
-  for (int item = item_lo; item < item_hi; ++item)
-    nstages += (bp.p[find_problem_by_item(bp, item)].k + 511) >> 9;
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     xsum[m] = 0;
@@ -319,9 +377,10 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
     for (int m = 0; m < MT; ++m)
 #pragma unroll
       for (int g = 0; g < 4; ++g) a[i][m][g] = 0;
-  for (int it = 0; it < nstages; ++it) {
-    const int s = it % S;
-    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / S) & 1, abort_flag))) break;
+  int s = 0;
+  uint32_t phase = 0;
+  while (true) {
+    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), phase, abort_flag))) break;
     StageMeta md;
     {
       const volatile int32_t* vm = reinterpret_cast<const volatile int32_t*>(meta + s);
@@ -330,6 +389,7 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
       md.kc = vm[2];
       md.info = vm[3];
     }
+    if (md.p < 0) break;  // the producer has no more work
     const int sw = (md.info >> 8) - 1;
     if (sw >= 0) {
       // A new problem: release the previous slot, take the new one.
@@ -410,6 +470,10 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));
+    if (++s == S) {
+      s = 0;
+      phase ^= 1u;
+    }
     if (md.info & 2) {
       // Tile done: add the 4 block lanes of each row, then
       // y = ((float)acc * xs[m]) * s.
@@ -450,6 +514,9 @@ struct QuantProblem {
 struct QuantBatchParams {
   int32_t count;
   int32_t m;
+  int32_t* queue;  // work counters of the decode launches that follow, zeroed here (or null)
+  int32_t nqueue;
+  int32_t pad;
   QuantProblem p[kQuantBatch];
 };
 
@@ -457,6 +524,9 @@ __global__ void __launch_bounds__(256) act_quant_batched_kernel(
     const __grid_constant__ QuantBatchParams qp) {
   grid_dependency_wait();
   grid_dependents_launch();
+  // The preceding grid (and so every earlier user of the counters) is done.
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < qp.nqueue; i += blockDim.x) qp.queue[i] = 0;
   __shared__ float red[32];
   const int p = blockIdx.x / qp.m;
   const int m = blockIdx.x % qp.m;

@@ -43,7 +43,8 @@ SIGNATURES = {
     "bitnet_i2s_quant_gemv": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bitnet_i2s_quant_gemv_batched_workspace_bytes": (_SZ, [_VP, _I32, _I64]),
     "bitnet_i2s_quant_gemv_batched": (_I32, [_VP, _I32, _I64, _VP, _SZ, _VP]),
-    "bitnet_i2s_gemv_batched": (_I32, [_VP, _I32, _I64, _VP]),
+    "bitnet_i2s_gemv_batched_workspace_bytes": (_SZ, [_I32]),
+    "bitnet_i2s_gemv_batched": (_I32, [_VP, _I32, _I64, _VP, _SZ, _VP]),
     "bitnet_i2s_quant_gemv_noalloc": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP]),
     "bitnet_debug_wait_timeout": (_I32, [_I64, _VP]),
     "bitnet_device_status": (_I32, []),
@@ -181,6 +182,10 @@ def bitnet_i2s_quant_gemv_workspace_bytes(m: int, k: int) -> int:
     return int(lib.bitnet_i2s_quant_gemv_workspace_bytes(m, k))
 
 
+def bitnet_i2s_gemv_batched_workspace_bytes(count: int) -> int:
+    return int(lib.bitnet_i2s_gemv_batched_workspace_bytes(count))
+
+
 def bitnet_i2s_quant_gemv(packed, n, k, x, y=None, acc=None, workspace=None, want_acc=False,
                           stream=None):
     """Per-token quantization of fp32 X[M,K] then the matmul: Y or (Y, acc)."""
@@ -262,9 +267,12 @@ class QProblem(ctypes.Structure):
 
 class BatchedGemv:
     """Argument block of one bitnet_i2s_gemv_batched call: a list of
-    (packed, N, K, Xq, xs, Y, acc_or_None) CUDA tensors, every Xq with M rows."""
+    (packed, N, K, Xq, xs, Y, acc_or_None) CUDA tensors, every Xq with M rows.
 
-    def __init__(self, problems, m: int):
+    `workspace`: True (default) allocates the work counters the call can use,
+    None passes no workspace (fixed tile ranges), or a uint8 CUDA tensor."""
+
+    def __init__(self, problems, m: int, workspace=True):
         self.m = int(m)
         self.tensors = []
         arr = (QProblem * len(problems))()
@@ -280,14 +288,23 @@ class BatchedGemv:
             self.tensors += [packed, xq, xs, y, acc]
         self.array = arr
         self.count = len(problems)
+        if workspace is True:
+            need = int(lib.bitnet_i2s_gemv_batched_workspace_bytes(self.count))
+            workspace = torch.empty(need, dtype=torch.uint8, device=problems[0][0].device)
+        if workspace is not None:
+            _need(workspace, "workspace", torch.uint8)
+        self.workspace = workspace
 
     def run(self, stream=None) -> None:
-        _check(lib.bitnet_i2s_gemv_batched(self.array, self.count, self.m, _stream(stream)))
+        ws = self.workspace
+        _check(lib.bitnet_i2s_gemv_batched(self.array, self.count, self.m,
+                                           None if ws is None else ws.data_ptr(),
+                                           0 if ws is None else ws.numel(), _stream(stream)))
 
 
-def bitnet_i2s_gemv_batched(problems, m: int, stream=None) -> None:
+def bitnet_i2s_gemv_batched(problems, m: int, workspace=True, stream=None) -> None:
     """One call for many independent (packed, N, K, Xq, xs, Y, acc) problems."""
-    BatchedGemv(problems, m).run(stream)
+    BatchedGemv(problems, m, workspace).run(stream)
 
 
 def bitnet_i2s_quant_gemv_noalloc(packed, n, k, x, y=None, acc=None, want_acc=False,

@@ -175,10 +175,13 @@ BITNET_API size_t bitnet_i2s_quant_gemv_batched_workspace_bytes(const bitnet_i2s
                                                                 int count, int64_t M);
 
 /* bitnet_i2s_quant_gemv for `count` independent problems that share the token
- * count M, as few launches as possible: for M <= 2 (K <= 8192) one launch
- * quantizes every problem's activations and one persistent launch streams
- * every problem's packed weights, so the whole batch (for example the 210
- * projections of a 30-layer BitNet b1.58 stack) keeps HBM busy end to end.
+ * count M, as few launches as possible: one launch quantizes every problem's
+ * activations; for M <= 2 (K <= 8192) persistent launches of up to 160
+ * problems stream the packed weights, handing 128-row tiles out through a
+ * work counter in the workspace (longest tiles first), so the whole batch
+ * (for example the 210 projections of a 30-layer BitNet b1.58 stack) keeps
+ * HBM busy end to end; other shapes go to tensor-core launches of up to 96
+ * problems.
  * Results are identical to calling bitnet_i2s_quant_gemv on each problem
  * [P5 section 5: per-token AbsMax quantization, then the ternary contraction].
  *   problems: HOST array of `count` descriptors, read during the call only.
@@ -201,14 +204,25 @@ typedef struct bitnet_i2s_qproblem {
   int32_t* acc_or_null;   /* M*N int32 or NULL */
 } bitnet_i2s_qproblem;
 
+/* Workspace bytes bitnet_i2s_gemv_batched can use (0 for count < 1). */
+BITNET_API size_t bitnet_i2s_gemv_batched_workspace_bytes(int count);
+
 /* bitnet_i2s_gemm on `count` independent problems sharing the token count M
- * (for example q, k and v on one quantized input), in one persistent launch
- * when M <= 2 and every K <= 8192, else one launch per problem.  Same
- * results as the single-problem call [P5 section 5 figure; P1 "How I2_S
- * Kernels Process the Format"].  `problems` is a HOST array read during the
- * call only; no workspace is needed. */
+ * (for example q, k and v on one quantized input), in persistent launches
+ * of up to 160 problems when M <= 2 and K <= 8192 (the integer-ALU kernel),
+ * and of up to 96 problems on the tensor-core kernel otherwise.  Same results
+ * as the single-problem call [P5 section 5 figure; P1 "How I2_S Kernels
+ * Process the Format"].  `problems` is a HOST array read during the call only.
+ *   workspace: NULL, or device scratch of at least
+ *     bitnet_i2s_gemv_batched_workspace_bytes(count) bytes, 256-byte aligned,
+ *     not shared with work that may run at the same time.  With it, the
+ *     integer-ALU launches hand out their tiles through work counters there
+ *     (zeroed on `stream` first), which evens out the SMs' finishing times;
+ *     without it each CTA takes a fixed range of tiles.  Results are the same
+ *     either way. */
 BITNET_API bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int count,
-                                                 int64_t M, void* stream);
+                                                 int64_t M, void* workspace,
+                                                 size_t workspace_bytes, void* stream);
 
 /* bitnet_i2s_quant_gemv without a caller-supplied workspace, for callers
  * that cannot allocate device memory: for example a plug-in that receives only

@@ -113,3 +113,20 @@ def test_product_package_never_touches_the_oracle():
 def test_debug_wait_timeout_rejects_out_of_range_on_host(i2s):
     assert i2s.lib.bitnet_debug_wait_timeout(10, None) == 1
     assert i2s.lib.bitnet_debug_wait_timeout(10 ** 10, None) == 1
+
+
+def test_gemv_batched_workspace_checks_on_host(i2s):
+    assert i2s.bitnet_i2s_gemv_batched_workspace_bytes(0) == 0
+    one = i2s.bitnet_i2s_gemv_batched_workspace_bytes(1)
+    assert one >= 4 and one % 256 == 0
+    assert i2s.bitnet_i2s_gemv_batched_workspace_bytes(161) >= 8
+
+    class QP(ctypes.Structure):
+        _fields_ = [("packed", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                    ("Xq", ctypes.c_void_p), ("xs", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+                    ("acc_or_null", ctypes.c_void_p)]
+    arr = (QP * 1)(QP(A, 8, 128, A, A, A, None))
+    fn = i2s.lib.bitnet_i2s_gemv_batched
+    assert fn(arr, 1, 1, A + 16, one, None) == 3
+    assert fn(arr, 1, 1, A, one - 1, None) == 1
+    assert "workspace" in i2s.bitnet_last_error()

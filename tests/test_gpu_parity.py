@@ -357,8 +357,9 @@ def test_stack_batched_all_layers_sampled(i2s, m):
         assert column_sum_identity(acc_h, torch.from_numpy(xq), t)
 
 
+@pytest.mark.parametrize("workspace", [True, None], ids=["work-counter", "fixed-ranges"])
 @pytest.mark.parametrize("m", [1, 2, 5])
-def test_gemv_batched_on_quantized_inputs(i2s, m):
+def test_gemv_batched_on_quantized_inputs(i2s, m, workspace):
     shapes = [(640, 2560), (640, 2560), (2560, 2560), (33, 6912), (130, 128)]
     cases, problems = [], []
     for i, (n, k) in enumerate(shapes):
@@ -368,11 +369,38 @@ def test_gemv_batched_on_quantized_inputs(i2s, m):
         problems.append((dev(torch.from_numpy(packed)), n, k, dev(torch.from_numpy(xq)),
                          dev(torch.from_numpy(xs)), y, acc))
         cases.append((packed, n, k, xq, xs))
-    i2s.bitnet_i2s_gemv_batched(problems, m)
+    i2s.bitnet_i2s_gemv_batched(problems, m, workspace=workspace)
     for (packed, n, k, xq, xs), pr in zip(cases, problems):
         y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
         assert_acc_equal(pr[6].cpu().numpy(), acc_ref)
         assert_y_close(pr[5].cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("workspace", [True, None], ids=["work-counter", "fixed-ranges"])
+def test_gemv_batched_many_problems_repeated_on_one_workspace(i2s, workspace):
+    """Two integer-ALU launches; with a workspace, its counters are zeroed by
+    every call, so repeating the call on the same workspace gives the same
+    results (every output is poisoned in between)."""
+    m = 1
+    shapes = [(40 + 97 * (i % 7), 128 * (1 + i % 5)) for i in range(170)]
+    cases, problems = [], []
+    for i, (n, k) in enumerate(shapes):
+        w, t, x, packed, xq, xs = _case(m, n, k, 8000 + i)
+        y = torch.empty((m, n), device="cuda")
+        acc = torch.empty((m, n), dtype=torch.int32, device="cuda")
+        problems.append((dev(torch.from_numpy(packed)), n, k, dev(torch.from_numpy(xq)),
+                         dev(torch.from_numpy(xs)), y, acc))
+        cases.append((packed, n, k, xq, xs))
+    plan = i2s.BatchedGemv(problems, m, workspace=workspace)
+    for _ in range(2):
+        for pr in problems:
+            pr[5].fill_(float("nan"))
+            pr[6].fill_(-1)
+        plan.run()
+        for (packed, n, k, xq, xs), pr in zip(cases, problems):
+            y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+            assert_acc_equal(pr[6].cpu().numpy(), acc_ref, f"{n}x{k}")
+            assert_y_close(pr[5].cpu().numpy(), y_ref, f"{n}x{k}")
 
 
 # ------------------------------------------------ dequant and ternarization
