@@ -733,14 +733,12 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
   if (st != BITNET_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* queue = static_cast<int32_t*>(workspace);
-  if (queue != nullptr) {
-    cudaError_t e = cudaMemsetAsync(queue, 0, queue_bytes(count), s);
-    if (e != cudaSuccess) return cuda_fail(e, "zeroing the work counters");
-  }
   // Decode-kernel problems in launches of at most kMaxBatch, tensor-core
   // problems in launches of at most kMmaBatch.  The first launch is
-  // ordinary, so all earlier work on the stream has finished once it
-  // starts; the later ones are dependent launches that start as SMs free up.
+  // ordinary, or, with work counters, the one-warp grid that zeroes them
+  // after waiting for all earlier work on the stream; either way nothing
+  // later starts before that work has finished.  The later launches are
+  // dependent launches that start as SMs free up.
   static thread_local BatchParamsT<kMaxBatch> bp;
   std::vector<int> small;
   std::vector<MmaProblem> big;
@@ -757,6 +755,21 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
   bool first = true;
   if (!small.empty()) {
     const size_t nchunks = (small.size() + kMaxBatch - 1) / kMaxBatch;
+    if (queue != nullptr) {
+      // A one-warp grid zeroes the counters once the work before this call is
+      // done; the first decode launch reads them after waiting for it.
+      cudaLaunchConfig_t cfg;
+      std::memset(&cfg, 0, sizeof(cfg));
+      cfg.gridDim = dim3(1);
+      cfg.blockDim = dim3(32);
+      cfg.stream = s;
+      cudaLaunchAttribute attr = pdl_attr(true);
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      cudaError_t e = cudaLaunchKernelEx(&cfg, zero_counters_kernel, queue,
+                                         static_cast<int32_t>(nchunks));
+      if (e != cudaSuccess) return cuda_fail(e, "launch of the counter reset");
+    }
     for (size_t c = 0; c < nchunks; ++c) {
       const size_t lo = small.size() * c / nchunks;
       const size_t hi = small.size() * (c + 1) / nchunks;
@@ -767,7 +780,8 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
         const bitnet_i2s_qproblem& q = problems[small[i]];
         bp.p[i - lo] = make_problem(q.packed, q.N, q.K, nullptr, q.Xq, q.xs, q.Y, q.acc_or_null);
       }
-      st = launch_dp4a(bp, s, /*pdl=*/!first, dev, /*wait=*/false);
+      const bool after_reset = queue != nullptr && c == 0;
+      st = launch_dp4a(bp, s, /*pdl=*/!first || after_reset, dev, /*wait=*/after_reset);
       if (st != BITNET_OK) return st;
       first = false;
     }

@@ -500,6 +500,14 @@ __global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm
   }
 }
 
+// Zeroes the work counters of the decode launches that follow, once the
+// preceding grid (and with it every earlier user of the counters) is done.
+__global__ void __launch_bounds__(32) zero_counters_kernel(int32_t* queue, int32_t n) {
+  grid_dependency_wait();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) queue[i] = 0;
+  grid_dependents_launch();
+}
+
 // Per-token absmax quantization of many problems' activations in one launch:
 // one CTA per (problem, token) row, the same arithmetic as act_quant_kernel.
 constexpr int kQuantBatch = 1000;

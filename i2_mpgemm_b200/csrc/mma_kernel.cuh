@@ -365,6 +365,19 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
     const int ut = (warp - 2) * 32 + lane;  // 0..127 among the unpackers
     bool ok = true;
     int chunk = 0, blk = 0, ii = 0;
+    // A slot store still in flight: it completes while the next block is
+    // unpacked, and only then is the slot handed to the MMA issuer.
+    bool pending = false;
+    int pend_t = 0;
+    auto finish_pending = [&]() {
+      if (pending) {
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull_bar(pend_t));
+        pending = false;
+      }
+    };
     for (int item = item_lo; item < item_hi && ok; ++item, ++ii) {
       int p, rt, tt;
       mma_item(bp, item, T, &p, &rt, &tt);
@@ -409,6 +422,7 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
           for (int g = 0; g < 4; ++g)
 #pragma unroll
             for (int i = 0; i < 8; ++i) a[8 * g + i] = unpack_word<kCodes>(wv[i], g);
+          finish_pending();
           if (blk >= C::kASlots) {
             ok = __all_sync(0xffffffffu,
                             mbar_wait(aempty_bar(t), ((blk >> 2) - 1) & 1, abort_flag));
@@ -416,10 +430,8 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
           }
           tc_fence_after();
           tmem_st_32x32b_x32(tmem + lane_base + C::kACol + 32u * t, a);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(afull_bar(t));
+          pending = true;
+          pend_t = t;
         }
         __syncwarp();
         if (ok && lane == 0) mbar_arrive(empty_bar(s));
@@ -442,6 +454,8 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
         if (lane == 0) mbar_arrive(dfull_bar(b));
       }
     }
+    if (ok) finish_pending();
+    tmem_st_wait();  // no store of this thread outlives it
   } else {
     // ---------------------------------------------------------- epilogue
     const int quarter = warp & 3;
