@@ -315,9 +315,10 @@ def matmul_kernel_time(i2s, torch, probs, reps: int = 20):
     plan = i2s.BatchedGemv([(p.packed, p.n, p.k, q, s, p.y, None)
                             for p, (q, s) in zip(probs, qs)], m)
     # The decode kernel takes up to DECODE_BATCH problems per launch (M <= 2,
-    # K <= 8192), the tensor-core kernel up to MMA_BATCH; the call also zeroes
+    # K <= 8192, or M = 1 with K <= 30720), the tensor-core kernel up to
+    # MMA_BATCH; the call also zeroes
     # the decode launches' work counters (one memset, inside the timed region).
-    small = [p for p in probs if m <= 2 and p.k <= 8192]
+    small = [p for p in probs if (m <= 2 and p.k <= 8192) or (m == 1 and p.k <= 30720)]
     launches = -(-len(small) // DECODE_BATCH) + -(-(len(probs) - len(small)) // MMA_BATCH)
     for _ in range(3):
         plan.run()
@@ -414,11 +415,54 @@ def workload_config(layers: int, m: int):
 
 # ----------------------------------------------------------------- extras
 
+def int8_gemm_tops(torch):
+    """Dense int8 GEMM throughput of the library GEMM behind torch._int_mm
+    (cuBLASLt) at 8192^3, best of 10 launches, or None where it is refused.
+    A measurement of the tensor-core peak only; nothing on the path uses it."""
+    n = 8192
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda")
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda")
+        for bb in (b.t().contiguous().t(), b):
+            try:
+                torch._int_mm(a, bb)
+                torch.cuda.synchronize()
+                break
+            except RuntimeError:
+                bb = None
+        if bb is None:
+            return None
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._int_mm(a, bb)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return 2.0 * n ** 3 / best / 1e9
+    except Exception:  # an unsupported build or device: no measured peak
+        return None
+
+
+def gpu_ternary(torch, n: int, k: int, seed: int):
+    """Seeded ternary weights drawn on the device (same distribution as the
+    host generator: -1/0/+1 with p = .25/.5/.25 times s ~ U(0.5, 2)), for the
+    timing-only large layer whose host generation would take minutes."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    r = torch.randint(0, 4, (n, k), generator=g, device="cuda", dtype=torch.int32)
+    s = 0.5 + 1.5 * torch.rand((), generator=g, device="cuda")
+    return ((r == 3).float() - (r == 0).float()) * s
+
+
 def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
     out = {}
-    # int8 dense tensor peak: the measured bf16 burst peak times the nominal
-    # int8/bf16 ratio of 2 (4.5 vs 2.25 dense POPS)
-    int8_tops = 2.0 * peaks["bf16_tflops"]
+    # int8 dense tensor peak: the library int8 GEMM measured here, else the
+    # measured bf16 burst peak times the nominal int8/bf16 ratio of 2
+    derived = 2.0 * peaks["bf16_tflops"]
+    measured = int8_gemm_tops(torch)
+    int8_tops = measured if measured else derived
     # the batch-1 stack as 210 separate fused calls (420 launches per step)
     g = capture(torch, lambda: stack_step(i2s, probs1))
     ms = time_replays(torch, g, max(5, steps // 2), 3)
@@ -456,7 +500,9 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
                                    "frac_of_int8_peak": round(tops / int8_tops, 4)}
             del g
     pre["int8_peak_TOPS"] = round(int8_tops, 1)
-    pre["int8_peak_source"] = f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 ratio)"
+    pre["int8_peak_source"] = ("measured: torch._int_mm 8192^3 best of 10" if measured else
+                               f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 ratio)")
+    pre["int8_peak_derived_TOPS"] = round(derived, 1)
     out["prefill_gemm"] = pre
     # single k_proj GEMV (640 x 2560, batch 1): one launch vs graph steady state
     w, _, _ = inputs.ternary_weights(640, 2560, inputs.seed_single())
@@ -466,6 +512,55 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
                                                          workspace=pr.ws))
     ms = time_replays(torch, g, 200, 10)
     out["k_proj_single"] = {"us_per_call": round(ms * 1000, 2), "note": "L2-resident (0.41 MB)"}
+    del g
+    # k_proj streamed: distinct copies of the packed tensor totalling more
+    # than 4x L2, one batched fused call per step
+    copies = int(4 * 126e6 / (640 * 2560 // 4)) + 1
+    xs_ = torch.empty((copies, 1, 2560), device="cuda").copy_(pr.x.view(1, 1, 2560).expand(copies, 1, 2560))
+    ys_ = torch.empty((copies, 1, 640), device="cuda")
+    pk = [pr.packed.clone() for _ in range(copies)]
+    plan = i2s.BatchedQuantGemv([(pk[i], 640, 2560, xs_[i], ys_[i], None) for i in range(copies)], 1)
+    g = capture(torch, plan.run)
+    ms = time_replays(torch, g, max(5, steps // 2), 3)
+    nbytes = copies * 640 * 2560 // 4
+    out["k_proj_streamed"] = {"copies": copies, "ms_per_step": round(ms, 4),
+                              "packed_GBps": round(nbytes / ms / 1e6, 1),
+                              "frac_of_hbm_measured": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    del g, plan, pk, xs_, ys_
+    torch.cuda.empty_cache()
+    # large BitNet-style layer (hidden 8192, ffn 28672): two device copies of
+    # its 7 projections (428 MB, more than 3x L2) at M = 1, and one at M = 64
+    large = inputs.projections_large()
+    packs = []
+    for idx, p in enumerate(large):
+        w = gpu_ternary(torch, p.n, p.k, inputs.seed_large(idx))
+        packs.append(i2s.bitnet_i2s_pack(w))
+        del w
+    torch.cuda.empty_cache()
+    layer_bytes = sum(p.n * p.k // 4 for p in large)
+    for m, ncopy in ((1, 2), (64, 1)):
+        probs, keep = [], []
+        for c in range(ncopy):
+            for idx, p in enumerate(large):
+                pk = packs[idx] if c == 0 else packs[idx].clone()
+                x = inputs.activations(m, p.k, inputs.seed_large(idx)).cuda()
+                y = torch.empty((m, p.n), device="cuda")
+                probs.append((pk, p.n, p.k, x, y, None))
+        plan = i2s.BatchedQuantGemv(probs, m)
+        g = capture(torch, plan.run)
+        ms = time_replays(torch, g, max(5, steps // 2), 3)
+        nbytes = ncopy * layer_bytes
+        ops = ncopy * sum(2.0 * m * p.n * p.k for p in large)
+        out[f"large_layer_M{m}"] = {
+            "layers": ncopy, "ms_per_step": round(ms, 4),
+            "packed_GBps": round(nbytes / ms / 1e6, 1),
+            "frac_of_hbm_measured": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
+            "TOPS": round(ops / ms / 1e9, 1), "frac_of_int8_peak": round(ops / ms / 1e9 / int8_tops, 4),
+            "tokens_per_s": round(m * 1000.0 / (ms / ncopy), 1)}
+        del g, plan, probs
+        torch.cuda.empty_cache()
+    del packs
+    torch.cuda.empty_cache()
     return out
 
 
@@ -525,6 +620,8 @@ def run_native(args):
     if rank == 0 and not args.no_extra:
         extra = extra_measurements(i2s, torch, inputs, args.steps, probs, peaks)
     extra["step_frac_of_hbm_peak"] = round(value / world / peaks["hbm_gbs"], 4)
+    extra["step_frac_of_hbm_spec_8tbs"] = round(value / world / 8000.0, 4)
+    extra["kernel_frac_of_hbm_spec_8tbs"] = round(achieved / 8000.0, 4)
     extra["tokens_per_s"] = round(world * m * 1000.0 / ms, 1)
 
     cpu = None

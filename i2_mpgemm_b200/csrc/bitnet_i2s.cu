@@ -163,7 +163,11 @@ constexpr int kMaxBatch = 160;  // problems per launch: the parameter block stay
 // With a work queue, the share of a decode launch's stages in fixed per-CTA
 // ranges; the rest is handed out at run time.
 constexpr double kStaticShare = 0.7;
-bool use_dp4a(int64_t m, int64_t k) { return m >= 1 && m <= 2 && k <= kGemvMaxK; }
+bool use_dp4a(int64_t m, int64_t k) {
+  return (m >= 1 && m <= 2 && k <= kGemvMaxK) || (m == 1 && k <= kGemvMaxKLong);
+}
+// Decode problems share a launch only with problems of the same variant.
+bool long_k(int64_t k) { return k > kGemvMaxK; }
 
 // Tensor maps, 128-row tiles and their stage counts for every problem.
 template <int CAP>
@@ -210,12 +214,12 @@ bitnet_status plan_items(BatchParamsT<CAP>& bp) {
   return BITNET_OK;
 }
 
-template <int MT, int CAP>
-bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, int grid, cudaStream_t stream, bool pdl,
-                            int dev) {
-  using C = GemvCfg<MT>;
+template <int MT, int CAP, int KMAX = kGemvMaxK>
+bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev) {
+  using C = GemvCfg<MT, KMAX>;
   static std::atomic<uint8_t> smem_done[kMaxDevices];
-  auto kern = i2s_gemv_dp4a_kernel<MT, CAP>;
+  auto kern = i2s_gemv_dp4a_kernel<MT, CAP, KMAX>;
+  const int grid = std::min(bp.total_items, C::kCtasPerSm * sm_count(dev));
   bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
   if (st != BITNET_OK) return st;
   cudaLaunchConfig_t cfg;
@@ -242,12 +246,11 @@ bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, 
   bitnet_status st = plan_items(bp);
   if (st != BITNET_OK) return st;
   bp.pdl = (pdl && wait) ? 1 : 0;
-  const int sms = sm_count(dev);
-  if (bp.m == 1)
-    return launch_dp4a_t<1, CAP>(bp, std::min(bp.total_items, GemvCfg<1>::kCtasPerSm * sms),
-                                 stream, pdl, dev);
-  return launch_dp4a_t<2, CAP>(bp, std::min(bp.total_items, GemvCfg<2>::kCtasPerSm * sms), stream,
-                               pdl, dev);
+  int kmax = 0;
+  for (int i = 0; i < bp.count; ++i) kmax = std::max(kmax, bp.p[i].k);
+  if (bp.m == 1 && long_k(kmax)) return launch_dp4a_t<1, CAP, kGemvMaxKLong>(bp, stream, pdl, dev);
+  if (bp.m == 1) return launch_dp4a_t<1, CAP>(bp, stream, pdl, dev);
+  return launch_dp4a_t<2, CAP>(bp, stream, pdl, dev);
 }
 
 BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const float* x,
@@ -392,9 +395,39 @@ constexpr int64_t kMaxTokens = int64_t{65535} * 16;  // grid.y limit at the smal
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
-// Work counters of the decode launches of a batch of `count` problems.
+// Work counters of the decode launches of a batch of `count` problems (the
+// two variants are chunked separately, hence at most one launch more).
 size_t queue_bytes(int count) {
-  return align256(sizeof(int32_t) * static_cast<size_t>((count + kMaxBatch - 1) / kMaxBatch));
+  return align256(sizeof(int32_t) * static_cast<size_t>((count + kMaxBatch - 1) / kMaxBatch + 1));
+}
+
+// Cuts the decode problems (indices into a batch; `nk_of(i)` gives problem
+// i's N and K) into launches of at most kMaxBatch problems, in chunks of
+// equal size.  A launch runs one kernel variant, chosen by its largest K.
+// When the long-K problems have fewer 128-row tiles than the long-K variant
+// keeps CTAs on the GPU, every problem joins them in that variant, so the
+// launch still has work for every CTA; otherwise the two kinds get separate
+// launches.
+template <typename NKOf>
+std::vector<std::pair<size_t, size_t>> decode_chunks(std::vector<int>& idx, NKOf nk_of, int dev) {
+  const auto mid = std::stable_partition(idx.begin(), idx.end(),
+                                         [&](int i) { return !long_k(nk_of(i).second); });
+  size_t split = static_cast<size_t>(mid - idx.begin());
+  int64_t long_tiles = 0;
+  for (size_t j = split; j < idx.size(); ++j)
+    long_tiles += (nk_of(idx[j]).first + kGemvTileRows - 1) / kGemvTileRows;
+  const int64_t long_ctas =
+      static_cast<int64_t>(GemvCfg<1, kGemvMaxKLong>::kCtasPerSm) * sm_count(dev);
+  if (split < idx.size() && long_tiles < long_ctas) split = 0;  // one group
+  std::vector<std::pair<size_t, size_t>> out;
+  for (const auto& g : {std::make_pair(size_t{0}, split), std::make_pair(split, idx.size())}) {
+    const size_t n = g.second - g.first;
+    if (n == 0) continue;
+    const size_t nchunks = (n + kMaxBatch - 1) / kMaxBatch;
+    for (size_t c = 0; c < nchunks; ++c)
+      out.emplace_back(g.first + n * c / nchunks, g.first + n * (c + 1) / nchunks);
+  }
+  return out;
 }
 
 }  // namespace
@@ -680,10 +713,11 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
   }
   bool first = true;
   if (!small.empty()) {
-    const size_t nchunks = (small.size() + kMaxBatch - 1) / kMaxBatch;
-    for (size_t c = 0; c < nchunks; ++c) {
-      const size_t lo = small.size() * c / nchunks;
-      const size_t hi = small.size() * (c + 1) / nchunks;
+    const auto chunks = decode_chunks(
+        small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev);
+    for (size_t c = 0; c < chunks.size(); ++c) {
+      const size_t lo = chunks[c].first;
+      const size_t hi = chunks[c].second;
       bp.count = static_cast<int32_t>(hi - lo);
       bp.m = static_cast<int32_t>(M);
       bp.queue = queue + c;
@@ -754,7 +788,9 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
   }
   bool first = true;
   if (!small.empty()) {
-    const size_t nchunks = (small.size() + kMaxBatch - 1) / kMaxBatch;
+    const auto chunks = decode_chunks(
+        small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev);
+    const size_t nchunks = chunks.size();
     if (queue != nullptr) {
       // A one-warp grid zeroes the counters once the work before this call is
       // done; the first decode launch reads them after waiting for it.
@@ -771,8 +807,8 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
       if (e != cudaSuccess) return cuda_fail(e, "launch of the counter reset");
     }
     for (size_t c = 0; c < nchunks; ++c) {
-      const size_t lo = small.size() * c / nchunks;
-      const size_t hi = small.size() * (c + 1) / nchunks;
+      const size_t lo = chunks[c].first;
+      const size_t hi = chunks[c].second;
       bp.count = static_cast<int32_t>(hi - lo);
       bp.m = static_cast<int32_t>(M);
       bp.queue = queue != nullptr ? queue + c : nullptr;

@@ -53,7 +53,8 @@
 namespace bitnet {
 
 constexpr int kGemvTileRows = 128;
-constexpr int kGemvMaxK = 8192;  // the x slot holds M x K bytes, K <= 8192
+constexpr int kGemvMaxK = 8192;      // the x slot holds M x K bytes, K <= 8192 ...
+constexpr int kGemvMaxKLong = 30720;  // ... or, in the one-token long-K variant, K <= 30720
 
 // One independent problem of a batch (device pointers and shape).
 struct BatchProblem {
@@ -90,16 +91,18 @@ struct StageMeta {
   int32_t info;  // bit 0: first box of the tile, bit 1: last box, bits 8..: switch index + 1
 };
 
-template <int MT>
+template <int MT, int KMAX = kGemvMaxK>
 struct GemvCfg {
   static_assert(MT >= 1 && MT <= 2, "tokens");
+  static_assert(KMAX == kGemvMaxK || (MT == 1 && KMAX == kGemvMaxKLong), "variant");
   static constexpr int kComputeWarps = kGemvTileRows / 32;
   static constexpr int kThreads = 32 * (kComputeWarps + 1);
   static constexpr int kBoxBytes = kGemvTileRows * 128;  // 16 KB
-  // One token: 3 stages and 3 CTAs per SM; two tokens: 4 stages, 2 CTAs.
+  // One token: 3 stages and 3 CTAs per SM (2 with the long-K activation
+  // slots); two tokens: 4 stages, 2 CTAs.
   static constexpr int kStages = MT == 1 ? 3 : 4;
-  static constexpr int kCtasPerSm = MT == 1 ? 3 : 2;
-  static constexpr int kXSlotBytes = MT * kGemvMaxK + 512;  // + slack read past K, never used
+  static constexpr int kCtasPerSm = (MT == 1 && KMAX == kGemvMaxK) ? 3 : 2;
+  static constexpr int kXSlotBytes = MT * KMAX + 512;  // + slack read past K, never used
   static constexpr int kBars = 2 * kStages + 4;
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kBoxBytes +
                                        2 * kXSlotBytes + kBars * 8 +
@@ -141,10 +144,10 @@ __device__ __forceinline__ int first_item_at_stage(const BP& bp, int target) {
   return off >= items ? P.item_start + items : P.item_start + off;
 }
 
-template <int MT, int CAP>
-__global__ void __launch_bounds__(GemvCfg<MT>::kThreads, GemvCfg<MT>::kCtasPerSm)
+template <int MT, int CAP, int KMAX = kGemvMaxK>
+__global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>::kCtasPerSm)
     i2s_gemv_dp4a_kernel(const __grid_constant__ BatchParamsT<CAP> bp) {
-  using C = GemvCfg<MT>;
+  using C = GemvCfg<MT, KMAX>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(

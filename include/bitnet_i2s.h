@@ -176,7 +176,8 @@ BITNET_API size_t bitnet_i2s_quant_gemv_batched_workspace_bytes(const bitnet_i2s
 
 /* bitnet_i2s_quant_gemv for `count` independent problems that share the token
  * count M, as few launches as possible: one launch quantizes every problem's
- * activations; for M <= 2 (K <= 8192) persistent launches of up to 160
+ * activations; for M = 1 with K <= 30720 and M = 2 with K <= 8192,
+ * persistent launches of up to 160
  * problems stream the packed weights, handing 128-row tiles out through a
  * work counter in the workspace (longest tiles first), so the whole batch
  * (for example the 210 projections of a 30-layer BitNet b1.58 stack) keeps
@@ -209,7 +210,8 @@ BITNET_API size_t bitnet_i2s_gemv_batched_workspace_bytes(int count);
 
 /* bitnet_i2s_gemm on `count` independent problems sharing the token count M
  * (for example q, k and v on one quantized input), in persistent launches
- * of up to 160 problems when M <= 2 and K <= 8192 (the integer-ALU kernel),
+ * of up to 160 problems when M = 1 with K <= 30720 or M = 2 with K <= 8192
+ * (the integer-ALU kernel),
  * and of up to 96 problems on the tensor-core kernel otherwise.  Same results
  * as the single-problem call [P5 section 5 figure; P1 "How I2_S Kernels
  * Process the Format"].  `problems` is a HOST array read during the call only.

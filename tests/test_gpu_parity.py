@@ -276,8 +276,10 @@ def test_no_device_wait_timed_out(i2s):
 
 # ------------------------------------------- decode ALU path and batching
 
-# M = 1, 2 with K <= 8192 run on the integer-ALU decode kernel.
+# M = 1 with K <= 30720 and M = 2 with K <= 8192 run on the integer-ALU
+# decode kernel (K > 8192 on its one-token long-K variant).
 DECODE = [(1, 1, 128), (1, 300, 2560), (2, 130, 640), (1, 129, 8192), (2, 257, 8192),
+          (1, 130, 8320), (1, 257, 28672), (1, 3, 30720),
           (2, 64, 4096), (1, 1000, 6912), (2, 7, 384)]
 
 
@@ -316,6 +318,26 @@ def test_batched_mixed_shapes(i2s, m):
         y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
         assert_acc_equal(acc.cpu().numpy(), acc_ref, f"{n}x{k}")
         assert_y_close(y.cpu().numpy(), y_ref, f"{n}x{k}")
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["quant-gemv", "gemv"])
+def test_batched_one_token_long_and_short_k(i2s, fused):
+    """One token: K <= 8192 and 8192 < K <= 30720 problems go to separate
+    launches of the two decode variants within one call."""
+    m = 1
+    shapes = [(130, 2560), (257, 28672), (7, 128), (33, 12288), (640, 2560), (65, 30720)]
+    cases, problems = _batched_problems(shapes, m, 5100)
+    if fused:
+        i2s.bitnet_i2s_quant_gemv_batched(problems, m)
+    else:
+        q = []
+        for (packed, n, k, xq, xs), (d_packed, _, _, _, y, acc) in zip(cases, problems):
+            q.append((d_packed, n, k, dev(torch.from_numpy(xq)), dev(torch.from_numpy(xs)), y, acc))
+        i2s.bitnet_i2s_gemv_batched(q, m)
+    for (packed, n, k, xq, xs), pr in zip(cases, problems):
+        y_ref, acc_ref = oracle.gemm(packed, n, k, xq, xs)
+        assert_acc_equal(pr[5].cpu().numpy(), acc_ref, f"{n}x{k}")
+        assert_y_close(pr[4].cpu().numpy(), y_ref, f"{n}x{k}")
 
 
 def test_batched_more_than_one_launch_worth_of_problems(i2s):
