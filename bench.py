@@ -370,6 +370,42 @@ def cpu_baseline(inputs, m: int, budget_s: float):
                       f"(scalar C oracle, one thread, {spent:.1f} s)"}
 
 
+_WORKER_SAMPLE = None
+
+
+def _oracle_worker_init(m: int):
+    global _WORKER_SAMPLE
+    from i2_mpgemm_b200 import inputs
+    _WORKER_SAMPLE = oracle_layer_sample(inputs, m)
+
+
+def _oracle_worker_task(idx: int) -> int:
+    import oracle
+    packed, n, k, x = _WORKER_SAMPLE[idx]
+    oracle.quant_gemm(packed, n, k, x)
+    return n * k // 4
+
+
+def cpu_baseline_all_cores(m: int, budget_s: float):
+    """The same oracle, one process per host core (spawned: the parent has a
+    CUDA context), each taking whole projections of the one-layer sample."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    cores = os.cpu_count() or 1
+    # A worker that dies raises here instead of being replaced forever.
+    with ProcessPoolExecutor(cores, mp_context=mp.get_context("spawn"),
+                             initializer=_oracle_worker_init, initargs=(m,)) as pool:
+        list(pool.map(_oracle_worker_task, list(range(7)) * cores))  # warm every worker
+        done, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < budget_s:
+            done += sum(pool.map(_oracle_worker_task, list(range(7)) * cores))
+        spent = time.perf_counter() - t0
+    return {"value": round(done / spent / 1e9, 6), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"rounds of {cores} x one layer's 7 projections at batch {m} over {cores} "
+                      f"spawned processes ({spent:.1f} s)"}
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -627,6 +663,8 @@ def run_native(args):
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_baseline(inputs, m, args.cpu_seconds)
+        if not args.no_extra:
+            extra["cpu_baseline_all_cores"] = cpu_baseline_all_cores(m, args.cpu_seconds / 2)
 
     cfg = workload_config(args.layers, m)
     cfg["packed_bytes_per_step"] = packed_bytes

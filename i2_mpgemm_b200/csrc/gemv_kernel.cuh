@@ -460,14 +460,16 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
         const uint4 w0 = *reinterpret_cast<const uint4*>(wrow + (((2 * cp) ^ rs) << 4));
         const uint4 w1 = *reinterpret_cast<const uint4*>(wrow + (((2 * cp + 1) ^ rs) << 4));
         const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        // Visit order: with two tokens, consecutive dp4a feed different
+        // accumulators (word-major), which measured about 3 % faster; one
+        // token keeps group-major order.
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int o = 0; o < 32; ++o) {
+          const int j = MT == 1 ? o / 8 : o % 4;
+          const int q = MT == 1 ? o % 8 : o / 4;
+          const uint32_t v = wv[q] & gmask[j];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint32_t v = wv[q] & gmask[j];
-#pragma unroll
-            for (int m = 0; m < MT; ++m) a[i][m][j] = dp4a_u8s8(v, xr[m][j][q], a[i][m][j]);
-          }
+          for (int m = 0; m < MT; ++m) a[i][m][j] = dp4a_u8s8(v, xr[m][j][q], a[i][m][j]);
         }
       }
     }

@@ -95,6 +95,7 @@ struct MmaCfg {
   static constexpr int kStages = (T <= 16) ? 4 : (T <= 32 ? 3 : 2);
   static constexpr int kCtasPerSm = (T <= 64) ? 2 : 1;
   static constexpr int kASlots = 4;
+  static constexpr int kAGroup = 2;  // A slots handed over per handshake (two groups in flight)
   static constexpr uint32_t kDCols = round32(T);        // one accumulator buffer
   static constexpr uint32_t kACol = 2 * kDCols;         // A slots after both buffers
   static constexpr uint32_t kTmemCols = pow2_at_least(kACol + 32u * kASlots);
@@ -332,11 +333,14 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
           const uint32_t xbase = smem_u32(smem + s * C::kStageBytes + C::kWTileBytes);
           for (int bi = 0; bi < nb; ++bi, ++blk) {
             const int t = blk & 3;
-            if (!mbar_wait(afull_bar(t), (blk >> 2) & 1, abort_flag)) {
-              ok = false;
-              break;
+            const int group = blk / C::kAGroup;
+            if (blk % C::kAGroup == 0) {
+              if (!mbar_wait(afull_bar(group & 1), (group >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
-            tc_fence_after();
             const uint32_t xb = xbase + bi * C::kXBoxBytes;
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
@@ -345,7 +349,7 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
                             smem_desc_sw128(xb + 32u * g), C::kIdesc, first ? 0u : 1u);
               first = false;
             }
-            tc_commit(aempty_bar(t));
+            if (blk % C::kAGroup == C::kAGroup - 1) tc_commit(aempty_bar(group & 1));
           }
           if (ok) tc_commit(empty_bar(s));
         }
@@ -365,18 +369,13 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
     const int ut = (warp - 2) * 32 + lane;  // 0..127 among the unpackers
     bool ok = true;
     int chunk = 0, blk = 0, ii = 0;
-    // A slot store still in flight: it completes while the next block is
-    // unpacked, and only then is the slot handed to the MMA issuer.
-    bool pending = false;
-    int pend_t = 0;
-    auto finish_pending = [&]() {
-      if (pending) {
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(afull_bar(pend_t));
-        pending = false;
-      }
+    // A slots are handed over in pairs (C::kAGroup blocks): one store wait
+    // and one arrival per pair, and one commit per pair on the MMA side.
+    auto hand_over = [&](int group) {
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(afull_bar(group & 1));
     };
     for (int item = item_lo; item < item_hi && ok; ++item, ++ii) {
       int p, rt, tt;
@@ -422,16 +421,16 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
           for (int g = 0; g < 4; ++g)
 #pragma unroll
             for (int i = 0; i < 8; ++i) a[8 * g + i] = unpack_word<kCodes>(wv[i], g);
-          finish_pending();
-          if (blk >= C::kASlots) {
+          const int group = blk / C::kAGroup;
+          if (blk % C::kAGroup == 0 && group >= 2) {
+            // The pair of slots this group reuses has been read by its MMAs.
             ok = __all_sync(0xffffffffu,
-                            mbar_wait(aempty_bar(t), ((blk >> 2) - 1) & 1, abort_flag));
+                            mbar_wait(aempty_bar(group & 1), ((group >> 1) - 1) & 1, abort_flag));
             if (!ok) break;
           }
           tc_fence_after();
           tmem_st_32x32b_x32(tmem + lane_base + C::kACol + 32u * t, a);
-          pending = true;
-          pend_t = t;
+          if (blk % C::kAGroup == C::kAGroup - 1) hand_over(group);
         }
         __syncwarp();
         if (ok && lane == 0) mbar_arrive(empty_bar(s));
@@ -454,7 +453,7 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
         if (lane == 0) mbar_arrive(dfull_bar(b));
       }
     }
-    if (ok) finish_pending();
+    if (ok && blk % C::kAGroup != 0) hand_over(blk / C::kAGroup);  // a last, partial pair
     tmem_st_wait();  // no store of this thread outlives it
   } else {
     // ---------------------------------------------------------- epilogue
