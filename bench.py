@@ -62,6 +62,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the gate 6912x2560 prefill GEMM at M=2048 (a small case "
+                         "for profiling the tensor-core kernel) and print its own line")
     return ap.parse_args(argv)
 
 
@@ -622,7 +625,11 @@ def run_native(args):
     packed_bytes = sum(p.packed_bytes for p in probs)
     plan = stack_batch(i2s, probs)
     dp4a = m <= 2
-    launches_per_step = 2 if dp4a else 2 * len(probs)  # quantize + matmul
+    # One quantizer launch per 1000 problems, decode launches of up to
+    # DECODE_BATCH problems, tensor-core launches of up to MMA_BATCH.
+    small = sum(1 for p in probs if (m <= 2 and p.k <= 8192) or (m == 1 and p.k <= 30720))
+    launches_per_step = (-(-len(probs) // 1000) + -(-small // DECODE_BATCH)
+                         + -(-(len(probs) - small) // MMA_BATCH))
 
     g = capture(torch, plan.run)
     with ClockSampler(gpu_uuid(torch, local_rank)) as clk:
@@ -695,10 +702,31 @@ def run_native(args):
     return 0
 
 
+def run_prefill_only(args):
+    """gate 6912x2560 x 2048 tokens on pre-quantized activations: one warm
+    call, `warmup` then `steps` graph replays."""
+    import torch
+
+    from i2_mpgemm_b200 import i2s, inputs
+    n, k, m = 6912, 2560, 2048
+    seed = inputs.seed_prefill(0)
+    w, _, _ = inputs.ternary_weights(n, k, seed)
+    packed = i2s.bitnet_i2s_pack(w.cuda())
+    xq, xs = i2s.bitnet_act_quant_i8(inputs.activations(m, k, seed).cuda())
+    y = torch.empty((m, n), device="cuda")
+    g = capture(torch, lambda: i2s.bitnet_i2s_gemm(packed, n, k, xq, xs, y=y))
+    ms = time_replays(torch, g, max(1, args.steps), max(1, args.warmup))
+    print(json.dumps({"workload": "prefill GEMM gate 6912x2560, M=2048", "us": round(ms * 1000, 2),
+                      "TOPS": round(2.0 * m * n * k / ms / 1e9, 1)}))
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.prefill_only:
+        return run_prefill_only(args)
     return run_native(args)
 
 
