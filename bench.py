@@ -46,7 +46,8 @@ NOMINAL_INT8_OVER_BF16 = 2.0  # 4.5 POPS int8 dense / 2.25 PFLOP/s bf16 dense
 DECODE_BATCH = 160  # problems per launch of the decode kernel
 MMA_BATCH = 96  # problems per launch of the tensor-core kernel
 TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "i2s_gemv_dp4a_stack_batch1.md")
-DECODE_SOURCE = os.path.join(ROOT, "i2_mpgemm_b200", "csrc", "gemv_kernel.cuh")
+DECODE_SOURCES = [os.path.join(ROOT, "i2_mpgemm_b200", "csrc", f)
+                  for f in ("gemv_kernel.cuh", "ptx.cuh")]
 
 
 # ------------------------------------------------------------------ setup
@@ -114,13 +115,27 @@ def load_peaks():
                 "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def code_digest(paths) -> str:
+    """sha256 of the code of the given sources with comments and blank lines
+    removed, so that a comment edit keeps a capture valid and a code edit
+    does not."""
+    import hashlib
+    import re
+    parts = []
+    for path in paths:
+        text = open(path).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        parts.append("\n".join(l.rstrip() for l in text.splitlines() if l.strip()))
+    return hashlib.sha256("\n".join(parts).encode()).hexdigest()
+
+
 def measured_traffic():
     """DRAM bytes per launch of the decode kernel from the committed ncu
-    summary, or None when the kernel's source changed since the capture."""
-    import hashlib
+    summary, or None when the kernel's code changed since the capture."""
     try:
         text = open(TRAFFIC_SUMMARY).read()
-        src = hashlib.sha256(open(DECODE_SOURCE, "rb").read()).hexdigest()
+        src = code_digest(DECODE_SOURCES)
     except OSError:
         return None
     vals = {}
@@ -128,7 +143,7 @@ def measured_traffic():
         if ":" in line and line.strip().startswith("- "):
             key, _, val = line.strip()[2:].partition(":")
             vals[key.strip()] = val.strip().strip("`")
-    if vals.get("kernel source sha256") != src:
+    if vals.get("kernel code sha256") != src:
         return None
     try:
         return int(vals["dram bytes per launch"])

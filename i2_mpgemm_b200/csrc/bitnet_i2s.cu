@@ -156,9 +156,9 @@ int sm_count(int dev) {
   return v;
 }
 
-// The integer-ALU kernel serves one or two tokens with K up to 8192 (the
-// activations of one problem sit in a shared-memory slot); everything else
-// goes to the tensor-core kernel.
+// The integer-ALU kernel serves two tokens with K up to 8192 and one token
+// with K up to 30720 (the activations of one problem sit in a shared-memory
+// slot); everything else goes to the tensor-core kernel.
 constexpr int kMaxBatch = 160;  // problems per launch: the parameter block stays under 32 KB
 // With a work queue, the share of a decode launch's stages in fixed per-CTA
 // ranges; the rest is handed out at run time.
@@ -166,7 +166,7 @@ constexpr double kStaticShare = 0.7;
 bool use_dp4a(int64_t m, int64_t k) {
   return (m >= 1 && m <= 2 && k <= kGemvMaxK) || (m == 1 && k <= kGemvMaxKLong);
 }
-// Decode problems share a launch only with problems of the same variant.
+// K above the short activation slot: the one-token long-K variant.
 bool long_k(int64_t k) { return k > kGemvMaxK; }
 
 // Tensor maps, 128-row tiles and their stage counts for every problem.

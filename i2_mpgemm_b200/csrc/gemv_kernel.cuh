@@ -1,5 +1,7 @@
 // gemv_kernel.cuh -- decode-shaped I2_S matmul (1 or 2 tokens) on the integer
 // ALU, for one or many independent problems in a single persistent launch.
+// Two activation-slot sizes: K <= 8192 (one or two tokens, 3 or 2 CTAs per
+// SM) and, for one token, K <= 30720 (2 CTAs per SM).
 //
 // At one or two tokens the ternary contraction ("LLM Quantization
 // Paradigms: FP8, AWQ, EXL2 & BitNet b1.58 in 2026", section 5 figure,
@@ -10,11 +12,15 @@
 //   * Work item = a tile of 128 rows of one problem over the whole K.
 //     The tile streams in stages of one TMA box of 128 rows x 128 bytes
 //     (512 weights of each row) written with the 128-byte swizzle.
-//   * Each CTA owns one contiguous range of items, balanced by bytes, so it
-//     changes problem only a few times per launch.  Warp 0 (one lane) is the
-//     producer; on a change of problem it also copies the problem's int8
-//     activations (M x K bytes) into one of two x slots and stages the two
-//     scales next to them.
+//   * Each CTA owns one contiguous range of items, balanced by stages, so it
+//     changes problem only a few times per launch.  With a work counter
+//     (batched calls with a workspace) the ranges cover the first part of
+//     the launch's stages and the remaining items are handed out one at a
+//     time as CTAs become free, which evens out when the CTAs finish.
+//     Warp 0 (one lane) is the producer; on a change of problem it also
+//     copies the problem's int8 activations (M x K bytes) into one of two x
+//     slots and stages the two scales next to them.  Weights are streamed
+//     with an evict-first L2 policy, so the activations stay in L2.
 //   * Warps 1..4 compute; warp w owns rows 32w..32w+31 of the tile.  Within
 //     a box, lane (rs, cp) = (lane / 4, lane % 4) owns I2_S block cp (32
 //     bytes, 128 weights) of the 4 rows 32w + rs + 8i, i = 0..3.  It loads
