@@ -44,7 +44,8 @@
 //     For prefill, where the unpack is amortised over 128 tokens.
 //
 // Pipelines: full/empty over the shared-memory stages (TMA -> unpack + MMA),
-// afull/aempty over four TMEM A slots (unpack -> MMA), dfull/dempty over two
+// afull/aempty over four TMEM A slots handed over in pairs (unpack -> MMA),
+// dfull/dempty over two
 // accumulator buffers (MMA + unpackers -> epilogue -> MMA).  Every wait is
 // bounded (ptx.cuh); there are no named barriers, so a timed-out wait can
 // never leave another warp stuck.
