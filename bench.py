@@ -45,6 +45,9 @@ FALLBACK_BF16_TFLOPS = 1590.0
 NOMINAL_INT8_OVER_BF16 = 2.0  # 4.5 POPS int8 dense / 2.25 PFLOP/s bf16 dense
 DECODE_BATCH = 160  # problems per launch of the decode kernel
 MMA_BATCH = 96  # problems per launch of the tensor-core kernel
+# (N, K) of the seven projections of one BitNet-b1.58-2B-4T block
+STACK_SHAPES = [(2560, 2560), (640, 2560), (640, 2560), (2560, 2560), (6912, 2560), (6912, 2560),
+                (2560, 6912)]
 TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "i2s_gemv_dp4a_stack_batch1.md")
 DECODE_SOURCES = [os.path.join(ROOT, "i2_mpgemm_b200", "csrc", f)
                   for f in ("gemv_kernel.cuh", "ptx.cuh")]
@@ -460,7 +463,7 @@ def workload_config(layers: int, m: int):
                      "(q/o 2560x2560, k/v 640x2560, gate/up 6912x2560, down 2560x6912), "
                      f"decode batch {m}, fused act-quant + I2_S matmul per projection"),
         "global_batch": m,
-        "packed_bytes_per_step": None,
+        "packed_bytes_per_step": layers * sum(n * k // 4 for n, k in STACK_SHAPES),
         "l2": "inputs larger than L2: each step streams all packed weights (521 MB for 30 "
               "layers) from HBM",
         "parallelism": "replicas (data parallel, no collective)",
