@@ -118,6 +118,16 @@ def load_peaks():
                 "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def step_launches(m: int, ks) -> int:
+    """Kernel launches of one batched fused call on problems with these K:
+    one quantizer launch per 1000 problems, decode launches of up to
+    DECODE_BATCH problems (M <= 2 with K <= 8192, or M = 1 with K <= 30720),
+    tensor-core launches of up to MMA_BATCH problems for the rest."""
+    ks = list(ks)
+    small = sum(1 for k in ks if (m <= 2 and k <= 8192) or (m == 1 and k <= 30720))
+    return -(-len(ks) // 1000) + -(-small // DECODE_BATCH) + -(-(len(ks) - small) // MMA_BATCH)
+
+
 def code_digest(paths) -> str:
     """sha256 of the code of the given sources with comments and blank lines
     removed, so that a comment edit keeps a capture valid and a code edit
@@ -643,11 +653,7 @@ def run_native(args):
     packed_bytes = sum(p.packed_bytes for p in probs)
     plan = stack_batch(i2s, probs)
     dp4a = m <= 2
-    # One quantizer launch per 1000 problems, decode launches of up to
-    # DECODE_BATCH problems, tensor-core launches of up to MMA_BATCH.
-    small = sum(1 for p in probs if (m <= 2 and p.k <= 8192) or (m == 1 and p.k <= 30720))
-    launches_per_step = (-(-len(probs) // 1000) + -(-small // DECODE_BATCH)
-                         + -(-(len(probs) - small) // MMA_BATCH))
+    launches_per_step = step_launches(m, [p.k for p in probs])
 
     g = capture(torch, plan.run)
     with ClockSampler(gpu_uuid(torch, local_rank)) as clk:

@@ -130,3 +130,15 @@ def test_gemv_batched_workspace_checks_on_host(i2s):
     assert fn(arr, 1, 1, A + 16, one, None) == 3
     assert fn(arr, 1, 1, A, one - 1, None) == 1
     assert "workspace" in i2s.bitnet_last_error()
+
+
+def test_batched_workspace_includes_the_work_counters(i2s):
+    ks = [2560, 2560, 2560, 2560, 2560, 2560, 6912] * 30
+    arr = (i2s.Problem * len(ks))()
+    for i, k in enumerate(ks):
+        arr[i] = i2s.Problem(A, 640, k, A, A, None)
+    slots = sum(i2s.bitnet_i2s_quant_gemv_workspace_bytes(1, k) for k in ks)
+    need = i2s.lib.bitnet_i2s_quant_gemv_batched_workspace_bytes(arr, len(ks), 1)
+    # one 256-byte block of counters (three decode launches at most) after the slots
+    assert need == slots + 256
+    assert i2s.lib.bitnet_i2s_quant_gemv_batched_workspace_bytes(arr, 0, 1) == 0

@@ -1,0 +1,63 @@
+"""Host-side logic of bench.py, without a GPU: the launch count it reports,
+the workload description it prints, and the rule that ties the recorded
+DRAM traffic to the kernel code it was captured on."""
+import importlib.util
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+STACK_KS = [2560, 2560, 2560, 2560, 2560, 2560, 6912] * 30
+
+
+def test_launches_per_step(bench):
+    # batch 1 and 2: one quantizer launch, two decode launches (210 / 160)
+    assert bench.step_launches(1, STACK_KS) == 3
+    assert bench.step_launches(2, STACK_KS) == 3
+    # batch 16: one quantizer launch, three tensor-core launches (210 / 96)
+    assert bench.step_launches(16, STACK_KS) == 4
+    # long K: one token stays on the decode kernel, two tokens do not
+    assert bench.step_launches(1, [28672]) == 2
+    assert bench.step_launches(2, [28672]) == 2
+    assert bench.step_launches(1, [131072]) == 2
+    assert bench.step_launches(1, [128] * 1001) == 2 + 7
+
+
+def test_workload_config_counts_the_stack(bench):
+    cfg = bench.workload_config(30, 1)
+    n_k = [(2560, 2560), (640, 2560), (640, 2560), (2560, 2560), (6912, 2560), (6912, 2560),
+           (2560, 6912)]
+    assert cfg["packed_bytes_per_step"] == 30 * sum(n * k // 4 for n, k in n_k) == 521011200
+
+
+def test_code_digest_ignores_comments_only(bench, tmp_path):
+    a = tmp_path / "a.cuh"
+    a.write_text("int f(int x) {  // one\n  return x + 1;\n}\n/* block\n comment */\n")
+    b = tmp_path / "b.cuh"
+    b.write_text("// header\n\nint f(int x) {\n  return x + 1;   \n}\n")
+    c = tmp_path / "c.cuh"
+    c.write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.code_digest([a]) == bench.code_digest([b])
+    assert bench.code_digest([a]) != bench.code_digest([c])
+
+
+def test_recorded_traffic_is_dropped_when_the_code_changes(bench, tmp_path, monkeypatch):
+    got = bench.measured_traffic()
+    assert got is None or (isinstance(got, int) and got > 0)
+    changed = []
+    for path in bench.DECODE_SOURCES:
+        dst = tmp_path / os.path.basename(path)
+        dst.write_text(open(path).read() + "\nstatic const int kChanged = 1;\n")
+        changed.append(str(dst))
+    monkeypatch.setattr(bench, "DECODE_SOURCES", changed)
+    assert bench.measured_traffic() is None
