@@ -564,7 +564,8 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
             ms = time_replays(torch, g, 20, 3)
             tops = 2.0 * m * n * k / ms / 1e9
             pre[f"{name}_M{m}"] = {"us": round(ms * 1000, 2), "TOPS": round(tops, 1),
-                                   "frac_of_int8_peak": round(tops / int8_tops, 4)}
+                                   "frac_of_int8_peak": round(tops / int8_tops, 4),
+                                   "frac_of_int8_spec_4500": round(tops / 4500.0, 4)}
             del g
     pre["int8_peak_TOPS"] = round(int8_tops, 1)
     pre["int8_peak_source"] = ("measured: torch._int_mm 8192^3 best of 10" if measured else
