@@ -310,8 +310,11 @@ def capture(torch, fn):
     return g
 
 
-def time_replays(torch, g, steps: int, warmup: int, before=None, after=None) -> float:
-    """Milliseconds per replay, CUDA events on the replay stream."""
+def time_replays(torch, g, steps: int, warmup: int, before=None, after=None,
+                 collective: bool = True) -> float:
+    """Milliseconds per replay, CUDA events on the replay stream.  With
+    `collective`, every rank must call it (barriers before and after);
+    rank-0-only measurements pass collective=False."""
     for _ in range(warmup):
         if before:
             before()
@@ -319,7 +322,8 @@ def time_replays(torch, g, steps: int, warmup: int, before=None, after=None) -> 
         if after:
             after()
     torch.cuda.synchronize()
-    barrier()
+    if collective:
+        barrier()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
@@ -332,7 +336,8 @@ def time_replays(torch, g, steps: int, warmup: int, before=None, after=None) -> 
     end.record()
     end.synchronize()
     torch.cuda.synchronize()
-    barrier()
+    if collective:
+        barrier()
     return start.elapsed_time(end) / steps
 
 
@@ -532,7 +537,7 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
     int8_tops = measured if measured else derived
     # the batch-1 stack as 210 separate fused calls (420 launches per step)
     g = capture(torch, lambda: stack_step(i2s, probs1))
-    ms = time_replays(torch, g, max(5, steps // 2), 3)
+    ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
     nbytes = sum(p.packed_bytes for p in probs1)
     out["stack_batch1_per_call"] = {"ms_per_step": round(ms, 4),
                                     "packed_GBps": round(nbytes / ms / 1e6, 1),
@@ -543,7 +548,7 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
         probs = build_stack(i2s, torch, inputs, 30, m, 0)
         plan = stack_batch(i2s, probs)
         g = capture(torch, plan.run)
-        ms = time_replays(torch, g, max(5, steps // 2), 3)
+        ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
         nbytes = sum(p.packed_bytes for p in probs)
         out[f"stack_batch{m}"] = {"ms_per_step": round(ms, 4), "packed_GBps": round(
             nbytes / ms / 1e6, 1), "tokens_per_s": round(m * 1000.0 / ms, 1)}
@@ -561,7 +566,7 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
             xq, xs = i2s.bitnet_act_quant_i8(x.cuda())
             y = torch.empty((m, n), device="cuda")
             g = capture(torch, lambda: i2s.bitnet_i2s_gemm(packed, n, k, xq, xs, y=y))
-            ms = time_replays(torch, g, 20, 3)
+            ms = time_replays(torch, g, 20, 3, collective=False)
             tops = 2.0 * m * n * k / ms / 1e9
             pre[f"{name}_M{m}"] = {"us": round(ms * 1000, 2), "TOPS": round(tops, 1),
                                    "frac_of_int8_peak": round(tops / int8_tops, 4),
@@ -578,7 +583,7 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
     pr = Problem(i2s, torch, 640, 2560, 1, w, x.cuda(), torch.empty((1, 640), device="cuda"))
     g = capture(torch, lambda: i2s.bitnet_i2s_quant_gemv(pr.packed, 640, 2560, pr.x, y=pr.y,
                                                          workspace=pr.ws))
-    ms = time_replays(torch, g, 200, 10)
+    ms = time_replays(torch, g, 200, 10, collective=False)
     out["k_proj_single"] = {"us_per_call": round(ms * 1000, 2), "note": "L2-resident (0.41 MB)"}
     del g
     # k_proj streamed: distinct copies of the packed tensor totalling more
@@ -589,7 +594,7 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
     pk = [pr.packed.clone() for _ in range(copies)]
     plan = i2s.BatchedQuantGemv([(pk[i], 640, 2560, xs_[i], ys_[i], None) for i in range(copies)], 1)
     g = capture(torch, plan.run)
-    ms = time_replays(torch, g, max(5, steps // 2), 3)
+    ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
     nbytes = copies * 640 * 2560 // 4
     out["k_proj_streamed"] = {"copies": copies, "ms_per_step": round(ms, 4),
                               "packed_GBps": round(nbytes / ms / 1e6, 1),
@@ -616,7 +621,7 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
                 probs.append((pk, p.n, p.k, x, y, None))
         plan = i2s.BatchedQuantGemv(probs, m)
         g = capture(torch, plan.run)
-        ms = time_replays(torch, g, max(5, steps // 2), 3)
+        ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
         nbytes = ncopy * layer_bytes
         ops = ncopy * sum(2.0 * m * p.n * p.k for p in large)
         out[f"large_layer_M{m}"] = {
@@ -684,8 +689,11 @@ def run_native(args):
                 "bytes_per_launch": int(k_bytes // k_launches),
                 "launch_us_mean": round(1000 * k_ms / k_launches, 3)}
 
+    # Secondary measurements: one process only (with more ranks the others
+    # would wait at the final barrier longer than the process-group timeout),
+    # and no collective inside.
     extra = {}
-    if rank == 0 and not args.no_extra:
+    if rank == 0 and world == 1 and not args.no_extra:
         extra = extra_measurements(i2s, torch, inputs, args.steps, probs, peaks)
     extra["step_frac_of_hbm_peak"] = round(value / world / peaks["hbm_gbs"], 4)
     extra["step_frac_of_hbm_spec_8tbs"] = round(value / world / 8000.0, 4)
