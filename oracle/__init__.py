@@ -59,8 +59,22 @@ def _load():
             lib.i2s_oracle_quant_gemm.argtypes = [vp, i64, i64, vp, i64, vp, vp, vp, vp]
             lib.i2s_oracle_ternarize_absmean.argtypes = [vp, i64, f64, vp, vp]
             lib.i2s_oracle_dequant_f32.argtypes = [vp, i64, i64, vp]
+            lib.i2s_oracle_iq2bn_bytes.restype = ctypes.c_size_t
+            lib.i2s_oracle_iq2bn_bytes.argtypes = [i64, i64]
+            lib.i2s_oracle_iq1bn_bytes.restype = ctypes.c_size_t
+            lib.i2s_oracle_iq1bn_bytes.argtypes = [i64, i64]
+            i32 = ctypes.c_int
+            lib.i2s_oracle_iq2bn_pack.argtypes = [vp, i64, i64, i32, vp]
+            lib.i2s_oracle_iq2bn_unpack.argtypes = [vp, i64, i64, i32, vp, vp]
+            lib.i2s_oracle_iq1bn_pack.argtypes = [vp, i64, i64, vp]
+            lib.i2s_oracle_iq1bn_unpack.argtypes = [vp, i64, i64, vp, vp]
+            lib.i2s_oracle_iq1bn_encode_byte.argtypes = [vp]
+            lib.i2s_oracle_iq1bn_trit.argtypes = [i32, i32]
+            lib.i2s_oracle_gemm_rows.argtypes = [vp, vp, i64, i64, vp, vp, i64, vp, vp]
             for name in ("pack", "unpack", "act_quant", "gemm", "gemm_sampled", "quant_gemm",
-                         "ternarize_absmean", "dequant_f32"):
+                         "ternarize_absmean", "dequant_f32", "iq2bn_pack", "iq2bn_unpack",
+                         "iq1bn_pack", "iq1bn_unpack", "iq1bn_encode_byte", "iq1bn_trit",
+                         "gemm_rows"):
                 getattr(lib, "i2s_oracle_" + name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -178,3 +192,78 @@ def dequant_f32(packed: np.ndarray, n: int, k: int) -> np.ndarray:
     out = np.zeros((n, k), dtype=np.float32)
     _check(_load().i2s_oracle_dequant_f32(_p(packed), n, k, _p(out)), "dequant_f32")
     return out
+
+
+# ---- block-64 formats (IQ2_BN, IQ2_BN_R4, IQ1_BN): readings R11-R14 of the
+# C file; their byte layouts are parity unpinned (the page elides them).
+
+def iq2bn_bytes(n: int, k: int) -> int:
+    """Size of an IQ2_BN or IQ2_BN_R4 tensor: N*K/4 code bytes + N row scales."""
+    return int(_load().i2s_oracle_iq2bn_bytes(n, k))
+
+
+def iq1bn_bytes(n: int, k: int) -> int:
+    """Size of an IQ1_BN tensor: 13 bytes per 64 weights + N row scales."""
+    return int(_load().i2s_oracle_iq1bn_bytes(n, k))
+
+
+def iq2bn_pack(w: np.ndarray, r4: bool = False) -> np.ndarray:
+    """fp32 W[N,K] -> IQ2_BN (or IQ2_BN_R4) bytes."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    out = np.zeros(iq2bn_bytes(n, k), dtype=np.uint8)
+    _check(_load().i2s_oracle_iq2bn_pack(_p(w), n, k, int(r4), _p(out)), "iq2bn_pack")
+    return out
+
+
+def iq2bn_unpack(p: np.ndarray, n: int, k: int, r4: bool = False):
+    """IQ2_BN (or IQ2_BN_R4) bytes -> (int8 T[N,K], fp32 row scales d[N])."""
+    p = _c(p, np.uint8)
+    t = np.zeros((n, k), dtype=np.int8)
+    d = np.zeros(n, dtype=np.float32)
+    _check(_load().i2s_oracle_iq2bn_unpack(_p(p), n, k, int(r4), _p(t), _p(d)), "iq2bn_unpack")
+    return t, d
+
+
+def iq1bn_pack(w: np.ndarray) -> np.ndarray:
+    """fp32 W[N,K] -> IQ1_BN bytes."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    out = np.zeros(iq1bn_bytes(n, k), dtype=np.uint8)
+    _check(_load().i2s_oracle_iq1bn_pack(_p(w), n, k, _p(out)), "iq1bn_pack")
+    return out
+
+
+def iq1bn_unpack(p: np.ndarray, n: int, k: int):
+    """IQ1_BN bytes -> (int8 T[N,K], fp32 row scales d[N])."""
+    p = _c(p, np.uint8)
+    t = np.zeros((n, k), dtype=np.int8)
+    d = np.zeros(n, dtype=np.float32)
+    _check(_load().i2s_oracle_iq1bn_unpack(_p(p), n, k, _p(t), _p(d)), "iq1bn_unpack")
+    return t, d
+
+
+def iq1bn_encode_byte(trits) -> int:
+    """The IQ1_BN byte of five trits (each 0, 1 or 2; the first most significant)."""
+    a = _c(np.asarray(trits), np.int32)
+    return int(_load().i2s_oracle_iq1bn_encode_byte(_p(a)))
+
+
+def iq1bn_trit(byte: int, j: int) -> int:
+    """Trit j (0..4) of an IQ1_BN byte, by multiply and shift."""
+    return int(_load().i2s_oracle_iq1bn_trit(int(byte), int(j)))
+
+
+def gemm_rows(t: np.ndarray, d: np.ndarray, xq: np.ndarray, xs: np.ndarray):
+    """(Y, acc) of ternary T[N,K] with row scales d[N] and Xq[M,K]."""
+    t = _c(t, np.int8)
+    d = _c(d, np.float32)
+    xq = _c(xq, np.int8)
+    xs = _c(xs, np.float32)
+    n, k = t.shape
+    m = xq.shape[0]
+    y = np.zeros((m, n), dtype=np.float32)
+    acc = np.zeros((m, n), dtype=np.int32)
+    _check(_load().i2s_oracle_gemm_rows(_p(t), _p(d), n, k, _p(xq), _p(xs), m, _p(y), _p(acc)),
+           "gemm_rows")
+    return y, acc

@@ -290,3 +290,186 @@ int i2s_oracle_dequant_f32(const uint8_t* packed, int64_t n, int64_t k, float* w
   }
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------
+ * The block-64 formats that "ik_llama.cpp 运行 BitNet b1.58 2B 模型实战" (§5.2,
+ * §5.3, §6) converts I2_S into: IQ2_BN (about 2 bits per weight), its 4-row
+ * interleaved variant IQ2_BN_R4, and IQ1_BN (1.625 bits per weight).  The
+ * page fixes the block of 64 weights (K must be a multiple of 64), the bit
+ * rates, the conversion chain I2_S -> f32 -> IQ2_BN (§5.1), that each row is
+ * quantized on its own, that R4 packs rows in groups of 4 with IQ2_BN's block
+ * structure, and that IQ1_BN is decoded with multiplies, adds and shifts.  It
+ * elides the bits inside a block, so the layouts below are readings, and
+ * their byte-level parity is unpinned by anything outside this file:
+ *   R11 IQ2_BN: a block of 64 weights is 16 bytes; weight j of the block sits
+ *       in byte j % 16, group g = j / 16, bits [7-2g : 6-2g], code = q + 1
+ *       (the I2_S grouping of R2 on 64-weight blocks).  Row n is K/64 blocks;
+ *       the tensor is N*K/4 code bytes followed by N fp32 row scales
+ *       d_n = max_k |W[n,k]|, and q = clip(round_half_away(W/d_n), -1, 1) as
+ *       in R4 with the row's scale (d_n = 0 gives code 1).
+ *   R12 IQ2_BN_R4: N a multiple of 4; block b of row 4G + r is stored at byte
+ *       ((G * (K/64) + b) * 4 + r) * 16, so the four rows' blocks b sit next
+ *       to each other; codes inside a block and the N row scales as R11.
+ *   R13 IQ1_BN: a block of 64 weights is 13 bytes: byte i < 12 holds the
+ *       trits t = q + 1 of weights 5i .. 5i+4, byte 12 those of weights
+ *       60 .. 63 (a fifth trit 0).  With v = sum_j t_j 3^(4-j) (the first
+ *       weight most significant) the byte stores ceil(256 v / 243); trit j is
+ *       ((byte * 3^j) mod 256) * 3 >> 8.  Row scales as R11.
+ *   R14 The matmul on these formats is R7 with the row's scale in place of
+ *       the tensor's: y = ((float)acc * xs[m]) * d_n.
+ */
+#define BN_BLOCK 64
+#define IQ2BN_BLOCK_BYTES 16
+#define IQ1BN_BLOCK_BYTES 13
+
+static int bn_shape_ok(int64_t n, int64_t k) { return n >= 1 && k >= 1 && k % BN_BLOCK == 0; }
+
+size_t i2s_oracle_iq2bn_bytes(int64_t n, int64_t k) { return (size_t)(n * k / 4 + 4 * n); }
+size_t i2s_oracle_iq1bn_bytes(int64_t n, int64_t k) {
+  return (size_t)(n * (k / BN_BLOCK) * IQ1BN_BLOCK_BYTES + 4 * n);
+}
+
+/* Row scales d_n = max_k |W[n,k]| (R11). */
+static void row_absmax(const float* w, int64_t n, int64_t k, float* d) {
+  for (int64_t r = 0; r < n; ++r) d[r] = absmax_f32(w + r * k, k);
+}
+
+/* Byte index and shift of weight (n, c) in IQ2_BN (R11) or IQ2_BN_R4 (R12). */
+static void iq2bn_locate(int64_t k_dim, int64_t n, int64_t c, int r4, int64_t* byte_index,
+                         int* shift) {
+  int64_t b = c / BN_BLOCK, j = c % BN_BLOCK;
+  int64_t nb = k_dim / BN_BLOCK;
+  int64_t block_base;
+  if (r4) block_base = (((n / 4) * nb + b) * 4 + (n % 4)) * IQ2BN_BLOCK_BYTES;
+  else block_base = (n * nb + b) * IQ2BN_BLOCK_BYTES;
+  *byte_index = block_base + j % IQ2BN_BLOCK_BYTES;
+  *shift = 6 - 2 * (int)(j / IQ2BN_BLOCK_BYTES);
+}
+
+/* Pack fp32 W[N,K] into IQ2_BN (r4 = 0) or IQ2_BN_R4 (r4 = 1). */
+int i2s_oracle_iq2bn_pack(const float* w, int64_t n, int64_t k, int r4, uint8_t* out) {
+  if (!w || !out) return ORC_BAD_ARG;
+  if (!bn_shape_ok(n, k) || (r4 && n % 4 != 0)) return ORC_BAD_SHAPE;
+  int64_t code_bytes = n * k / 4;
+  memset(out, 0, (size_t)code_bytes);
+  float* d = (float*)(out + code_bytes); /* 4-byte aligned when out is */
+  float* dtmp = (float*)malloc((size_t)n * sizeof(float));
+  if (!dtmp) return ORC_BAD_ARG;
+  row_absmax(w, n, k, dtmp);
+  for (int64_t r = 0; r < n; ++r) {
+    for (int64_t c = 0; c < k; ++c) {
+      int code = ternary_of(w[r * k + c], dtmp[r]) + 1;
+      int64_t bi;
+      int sh;
+      iq2bn_locate(k, r, c, r4, &bi, &sh);
+      out[bi] = (uint8_t)(out[bi] | (code << sh));
+    }
+  }
+  memcpy(d, dtmp, (size_t)n * sizeof(float));
+  free(dtmp);
+  return ORC_OK;
+}
+
+/* IQ2_BN or IQ2_BN_R4 -> int8 T[N,K] and the row scales d[N]. */
+int i2s_oracle_iq2bn_unpack(const uint8_t* p, int64_t n, int64_t k, int r4, int8_t* t, float* d) {
+  if (!p || !t) return ORC_BAD_ARG;
+  if (!bn_shape_ok(n, k) || (r4 && n % 4 != 0)) return ORC_BAD_SHAPE;
+  for (int64_t r = 0; r < n; ++r) {
+    for (int64_t c = 0; c < k; ++c) {
+      int64_t bi;
+      int sh;
+      iq2bn_locate(k, r, c, r4, &bi, &sh);
+      int code = (p[bi] >> sh) & 3;
+      if (code == 3) return ORC_BAD_CODE;
+      t[r * k + c] = (int8_t)(code - 1);
+    }
+  }
+  if (d) memcpy(d, p + n * k / 4, (size_t)n * sizeof(float));
+  return ORC_OK;
+}
+
+/* The IQ1_BN byte of five trits t[0..4] (R13). */
+static uint8_t iq1bn_encode(const int* t) {
+  int v = 0;
+  for (int j = 0; j < 5; ++j) v = 3 * v + t[j];
+  return (uint8_t)((256 * v + 242) / 243); /* ceil(256 v / 243) */
+}
+
+/* Trit j (0..4) of an IQ1_BN byte (R13). */
+static int iq1bn_trit(uint8_t q, int j) {
+  int p3 = 1;
+  for (int i = 0; i < j; ++i) p3 *= 3;
+  return ((((int)q * p3) & 255) * 3) >> 8;
+}
+
+int i2s_oracle_iq1bn_encode_byte(const int* trits) { return iq1bn_encode(trits); }
+int i2s_oracle_iq1bn_trit(int byte, int j) { return iq1bn_trit((uint8_t)byte, j); }
+
+/* Pack fp32 W[N,K] into IQ1_BN (R13). */
+int i2s_oracle_iq1bn_pack(const float* w, int64_t n, int64_t k, uint8_t* out) {
+  if (!w || !out) return ORC_BAD_ARG;
+  if (!bn_shape_ok(n, k)) return ORC_BAD_SHAPE;
+  int64_t nb = k / BN_BLOCK;
+  int64_t code_bytes = n * nb * IQ1BN_BLOCK_BYTES;
+  float* d = (float*)malloc((size_t)n * sizeof(float));
+  if (!d) return ORC_BAD_ARG;
+  row_absmax(w, n, k, d);
+  for (int64_t r = 0; r < n; ++r) {
+    for (int64_t b = 0; b < nb; ++b) {
+      uint8_t* blk = out + (r * nb + b) * IQ1BN_BLOCK_BYTES;
+      for (int i = 0; i < IQ1BN_BLOCK_BYTES; ++i) {
+        int t[5] = {0, 0, 0, 0, 0};
+        for (int j = 0; j < 5; ++j) {
+          int e = 5 * i + j; /* weight of the block */
+          if (e < BN_BLOCK) t[j] = ternary_of(w[r * k + b * BN_BLOCK + e], d[r]) + 1;
+        }
+        blk[i] = iq1bn_encode(t);
+      }
+    }
+  }
+  memcpy(out + code_bytes, d, (size_t)n * sizeof(float));
+  free(d);
+  return ORC_OK;
+}
+
+/* IQ1_BN -> int8 T[N,K] and the row scales d[N] (R13). */
+int i2s_oracle_iq1bn_unpack(const uint8_t* p, int64_t n, int64_t k, int8_t* t, float* d) {
+  if (!p || !t) return ORC_BAD_ARG;
+  if (!bn_shape_ok(n, k)) return ORC_BAD_SHAPE;
+  int64_t nb = k / BN_BLOCK;
+  for (int64_t r = 0; r < n; ++r) {
+    for (int64_t b = 0; b < nb; ++b) {
+      const uint8_t* blk = p + (r * nb + b) * IQ1BN_BLOCK_BYTES;
+      for (int e = 0; e < BN_BLOCK; ++e) {
+        int tr = iq1bn_trit(blk[e / 5], e % 5);
+        if (tr > 2) return ORC_BAD_CODE;
+        t[r * k + b * BN_BLOCK + e] = (int8_t)(tr - 1);
+      }
+    }
+  }
+  if (d) memcpy(d, p + n * nb * IQ1BN_BLOCK_BYTES, (size_t)n * sizeof(float));
+  return ORC_OK;
+}
+
+/* Y[M,N] from ternary T[N,K] with row scales d[N] (R14: R7 with d_n). */
+int i2s_oracle_gemm_rows(const int8_t* t, const float* d, int64_t n, int64_t k,
+                         const int8_t* xq, const float* xs, int64_t m, float* y, int32_t* acc) {
+  if (!t || !d || !xq || !xs) return ORC_BAD_ARG;
+  if (n < 1 || k < 1 || m < 1) return ORC_BAD_SHAPE;
+  for (int64_t r = 0; r < m; ++r) {
+    for (int64_t c = 0; c < n; ++c) {
+      int32_t a = 0;
+      for (int64_t i = 0; i < k; ++i) {
+        int w = t[c * k + i];
+        if (w == 1) a += (int32_t)xq[r * k + i];
+        else if (w == -1) a -= (int32_t)xq[r * k + i];
+      }
+      if (acc) acc[r * n + c] = a;
+      if (y) {
+        float v = (float)a * xs[r];
+        y[r * n + c] = v * d[c];
+      }
+    }
+  }
+  return ORC_OK;
+}
