@@ -15,6 +15,7 @@
 #include <vector>
 
 #include "bitnet_i2s.h"
+#include "bn_kernels.cuh"
 #include "gemv_kernel.cuh"
 #include "mma_kernel.cuh"
 #include "quant_kernels.cuh"
@@ -160,6 +161,7 @@ int sm_count(int dev) {
 // with K up to 30720 (the activations of one problem sit in a shared-memory
 // slot); everything else goes to the tensor-core kernel.
 constexpr int kMaxBatch = 160;  // problems per launch: the parameter block stays under 32 KB
+static_assert(sizeof(BatchParamsT<kMaxBatch>) <= 32764, "decode kernel parameter block");
 // With a work queue, the share of a decode launch's stages in fixed per-CTA
 // ranges; the rest is handed out at run time.
 constexpr double kStaticShare = 0.7;
@@ -169,15 +171,56 @@ bool use_dp4a(int64_t m, int64_t k) {
 // K above the short activation slot: the one-token long-K variant.
 bool long_k(int64_t k) { return k > kGemvMaxK; }
 
-// Tensor maps, 128-row tiles and their stage counts for every problem.
+// Split K of the decode kernel: at most this many (slice, row tile) items
+// per launch, whose partial sums and arrival counters the workspace holds.
+constexpr int64_t kSplitItemsMax = 512;
+
+// Workspace ints of one decode launch's split area for `mt` tokens: the
+// arrival counters (zeroed before the launch), then the partial sums.
+size_t split_cnt_ints() { return static_cast<size_t>(kSplitItemsMax) * 4; }
+size_t split_part_ints(int64_t mt) { return static_cast<size_t>(kSplitItemsMax) * 128 * mt; }
+
+// K slices for the problems of one decode launch on `grid` CTAs.  When the
+// launch has fewer 128-row tiles than CTAs, every problem's K range is cut
+// into up to ceil(grid / tiles) slices of whole 512-wide boxes, keeping the
+// launch's items within kSplitItemsMax, so that the launch has work for
+// every CTA.
 template <int CAP>
-bitnet_status plan_items(BatchParamsT<CAP>& bp) {
+void plan_splits(BatchParamsT<CAP>& bp, int64_t grid) {
+  int64_t tiles = 0;
+  for (int i = 0; i < bp.count; ++i) tiles += (bp.p[i].n + kGemvTileRows - 1) / kGemvTileRows;
+  int64_t want = 1;
+  if (bp.split_base != nullptr && tiles < grid)
+    want = std::min((grid + tiles - 1) / tiles, kSplitItemsMax / tiles);
+  int64_t part = 0, cnt = 0;
+  for (int i = 0; i < bp.count; ++i) {
+    BatchProblem& q = bp.p[i];
+    const int64_t nk = (q.k + 511) / 512;
+    int64_t sp = std::max<int64_t>(1, std::min(want, nk));
+    const int64_t cps = (nk + sp - 1) / sp;
+    sp = (nk + cps - 1) / cps;
+    q.splits = static_cast<int32_t>(sp);
+    q.cps = static_cast<int32_t>(cps);
+    q.part_off = static_cast<int32_t>(part);
+    q.cnt_off = static_cast<int32_t>(cnt);
+    if (sp > 1) {
+      const int64_t t = (q.n + kGemvTileRows - 1) / kGemvTileRows;
+      part += t * sp * bp.m * 128;
+      cnt += t * 4;
+    }
+  }
+}
+
+// Tensor maps, work items and their stage counts for every problem.
+template <int CAP>
+bitnet_status plan_items(BatchParamsT<CAP>& bp, int64_t grid) {
   if (bp.queue != nullptr) {
     // Items are handed out in order: the longest ones (largest K) first, so
     // that the last items taken are short and the CTAs end together.
     std::stable_sort(bp.p, bp.p + bp.count,
                      [](const BatchProblem& a, const BatchProblem& b) { return a.k > b.k; });
   }
+  plan_splits(bp, grid);
   int64_t items = 0, stages = 0;
   for (int i = 0; i < bp.count; ++i) {
     BatchProblem& q = bp.p[i];
@@ -187,8 +230,8 @@ bitnet_status plan_items(BatchParamsT<CAP>& bp) {
     q.item_start = static_cast<int32_t>(items);
     q.stage_start = static_cast<int32_t>(stages);
     const int64_t tiles = (q.n + kGemvTileRows - 1) / kGemvTileRows;
-    items += tiles;
-    stages += tiles * ((q.k + 511) / 512);
+    items += tiles * q.splits;
+    stages += tiles * q.splits * q.cps;
     if (stages > int64_t{0x7fffffff}) return fail(BITNET_ERR_SHAPE, "too many rows in one batch");
   }
   bp.total_items = static_cast<int32_t>(items);
@@ -201,8 +244,8 @@ bitnet_status plan_items(BatchParamsT<CAP>& bp) {
     const int64_t cut = static_cast<int64_t>(kStaticShare * static_cast<double>(stages));
     for (int i = 0; i < bp.count; ++i) {
       const BatchProblem& q = bp.p[i];
-      const int64_t nk = (q.k + 511) / 512;
-      const int64_t tiles = (q.n + kGemvTileRows - 1) / kGemvTileRows;
+      const int64_t nk = q.cps;
+      const int64_t tiles = ((q.n + kGemvTileRows - 1) / kGemvTileRows) * q.splits;
       if (q.stage_start + tiles * nk > cut) {
         const int64_t off = std::max<int64_t>(0, (cut - q.stage_start + nk - 1) / nk);
         bp.dyn_start = static_cast<int32_t>(q.item_start + std::min(off, tiles));
@@ -215,12 +258,14 @@ bitnet_status plan_items(BatchParamsT<CAP>& bp) {
 }
 
 template <int MT, int CAP, int KMAX = kGemvMaxK>
-bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev) {
+bitnet_status launch_dp4a_t(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev) {
   using C = GemvCfg<MT, KMAX>;
   static std::atomic<uint8_t> smem_done[kMaxDevices];
   auto kern = i2s_gemv_dp4a_kernel<MT, CAP, KMAX>;
+  bitnet_status st = plan_items(bp, int64_t{C::kCtasPerSm} * sm_count(dev));
+  if (st != BITNET_OK) return st;
   const int grid = std::min(bp.total_items, C::kCtasPerSm * sm_count(dev));
-  bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
+  st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
   if (st != BITNET_OK) return st;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
@@ -243,8 +288,6 @@ bitnet_status launch_dp4a_t(const BatchParamsT<CAP>& bp, cudaStream_t stream, bo
 template <int CAP>
 bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev,
                           bool wait = true) {
-  bitnet_status st = plan_items(bp);
-  if (st != BITNET_OK) return st;
   bp.pdl = (pdl && wait) ? 1 : 0;
   int kmax = 0;
   for (int i = 0; i < bp.count; ++i) kmax = std::max(kmax, bp.p[i].k);
@@ -253,11 +296,10 @@ bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, 
   return launch_dp4a_t<2, CAP>(bp, stream, pdl, dev);
 }
 
-BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const float* x,
-                          const int8_t* xq, const float* xs, float* y, int32_t* acc) {
+BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const int8_t* xq,
+                          const float* xs, float* y, int32_t* acc) {
   BatchProblem q;
   q.packed = packed;
-  q.x = x;
   q.xq = const_cast<int8_t*>(xq);
   q.xs = const_cast<float*>(xs);
   q.y = y;
@@ -266,11 +308,16 @@ BatchProblem make_problem(const uint8_t* packed, int64_t n, int64_t k, const flo
   q.k = static_cast<int32_t>(k);
   q.item_start = 0;
   q.stage_start = 0;
+  q.splits = 1;
+  q.cps = static_cast<int32_t>((k + 511) / 512);
+  q.part_off = 0;
+  q.cnt_off = 0;
   return q;
 }
 
 // ------------------------------------------------------ tensor-core path
 constexpr int kMmaBatch = 96;  // problems per launch: the parameter block stays under 32 KB
+static_assert(sizeof(MmaParamsT<kMmaBatch>) <= 32764, "tensor-core kernel parameter block");
 
 // Tensor maps and item/chunk numbering for every problem of a batch.
 template <int T, int CAP>
@@ -356,7 +403,9 @@ bitnet_status run_matmul(const uint8_t* packed, int64_t n, int64_t k, const int8
     bp.count = 1;
     bp.m = static_cast<int32_t>(m);
     bp.queue = nullptr;
-    bp.p[0] = make_problem(packed, n, k, nullptr, xq, xs, y, acc);
+    bp.split_base = nullptr;
+    bp.cnt_base = nullptr;
+    bp.p[0] = make_problem(packed, n, k, xq, xs, y, acc);
     return launch_dp4a(bp, stream, pdl, dev);
   }
   MmaParamsT<1> bp;
@@ -395,10 +444,65 @@ constexpr int64_t kMaxTokens = int64_t{65535} * 16;  // grid.y limit at the smal
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
-// Work counters of the decode launches of a batch of `count` problems (the
-// two variants are chunked separately, hence at most one launch more).
-size_t queue_bytes(int count) {
-  return align256(sizeof(int32_t) * static_cast<size_t>((count + kMaxBatch - 1) / kMaxBatch + 1));
+// Workspace of one problem's quantized activations: M x K int8, then M
+// fp32 scales.
+size_t slot_bytes(int64_t m, int64_t k) {
+  return align256(static_cast<size_t>(m) * static_cast<size_t>(k)) +
+         align256(static_cast<size_t>(m) * sizeof(float));
+}
+
+// Decode launches of a batch of `count` problems at most (the two kernel
+// variants are chunked separately, hence one launch more when there are two
+// problems or more).
+size_t decode_launches(int count) {
+  return static_cast<size_t>((count + kMaxBatch - 1) / kMaxBatch + (count > 1 ? 1 : 0));
+}
+
+// The workspace after the activation slots: per decode launch a work
+// counter; for up to two tokens also per launch the split arrival counters
+// (all of them zeroed before the launches), then the split partial sums.
+size_t decode_tail_bytes(int count, int64_t m) {
+  const size_t nl = decode_launches(count);
+  const bool split = m <= 2;
+  size_t b = align256(sizeof(int32_t) * (nl + (split ? nl * split_cnt_ints() : 0)));
+  if (split) b += align256(sizeof(int32_t) * nl * split_part_ints(m));
+  return b;
+}
+
+struct DecodeTail {
+  int32_t* zero = nullptr;   // counters to zero before the decode launches
+  size_t zero_ints = 0;
+  int32_t* queue = nullptr;  // per launch: work counter
+  int32_t* cnt = nullptr;    // per launch: split_cnt_ints() arrival counters
+  int32_t* part = nullptr;   // per launch: split_part_ints(m) partial sums
+  int64_t m = 0;
+
+  template <int CAP>
+  void assign(BatchParamsT<CAP>& bp, size_t launch) const {
+    bp.queue = queue != nullptr ? queue + launch : nullptr;
+    bp.cnt_base = cnt != nullptr ? cnt + launch * split_cnt_ints() : nullptr;
+    bp.split_base = part != nullptr ? part + launch * split_part_ints(m) : nullptr;
+  }
+};
+
+// The decode tail at `base` (null: no workspace) for `count` problems of at
+// most `m` tokens.
+DecodeTail decode_tail(void* base, int count, int64_t m) {
+  DecodeTail t;
+  if (base == nullptr) return t;
+  const size_t nl = decode_launches(count);
+  const bool split = m <= 2;
+  int32_t* w = static_cast<int32_t*>(base);
+  t.zero = w;
+  t.zero_ints = nl + (split ? nl * split_cnt_ints() : 0);
+  t.queue = w;
+  if (split) {
+    t.cnt = w + nl;
+    t.part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(base) +
+                                        align256(sizeof(int32_t) * t.zero_ints));
+    t.m = m;
+  }
+  return t;
 }
 
 // Cuts the decode problems (indices into a batch; `nk_of(i)` gives problem
@@ -428,6 +532,99 @@ std::vector<std::pair<size_t, size_t>> decode_chunks(std::vector<int>& idx, NKOf
       out.emplace_back(g.first + n * c / nchunks, g.first + n * (c + 1) / nchunks);
   }
   return out;
+}
+
+// Quantizer launch(es) and matmul launches of a batch of fused problems on a
+// workspace laid out as bitnet_i2s_quant_gemv_batched_workspace_bytes says:
+// the problems' activation slots, then the decode tail.
+//  1. One launch quantizes every problem's tokens into the workspace (and
+//     zeroes the decode launches' counters).
+//  2. Problems the integer-ALU decode kernel serves (M <= 2, K <= 8192, or
+//     M = 1 with K <= 30720) run in launches of at most kMaxBatch problems,
+//     the rest in launches of at most kMmaBatch problems on the tensor-core
+//     kernel.
+// The first matmul launch waits for the quantizer; every later one is a
+// dependent launch that skips the wait and starts streaming as soon as SMs
+// free up: each launch in the chain starts only after every thread of the
+// one before it has signalled, which the first launch's threads do only
+// after their wait, so all of them start after the quantizer has finished;
+// no matmul writes what another reads; and every CTA waits for the grid
+// before its own before it exits, so the last launch completes last.
+bitnet_status run_quant_batched(const bitnet_i2s_problem* problems, int count, int64_t M,
+                                void* workspace, cudaStream_t s, int dev) {
+  static thread_local QuantBatchParams qp;         // 32 KB: kept off the stack
+  static thread_local BatchParamsT<kMaxBatch> bp;  // 32 KB
+  std::vector<std::pair<int8_t*, float*>> sl(static_cast<size_t>(count));
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  for (int i = 0; i < count; ++i) {
+    sl[i] = {reinterpret_cast<int8_t*>(w),
+             reinterpret_cast<float*>(w + align256(static_cast<size_t>(M) * problems[i].K))};
+    w += slot_bytes(M, problems[i].K);
+  }
+  const DecodeTail tail = decode_tail(w, count, M);
+  for (int base = 0; base < count; base += kQuantBatch) {
+    const int cnt = std::min(kQuantBatch, count - base);
+    qp.count = cnt;
+    qp.m = static_cast<int32_t>(M);
+    // The first quantizer launch zeroes the counters; every decode launch
+    // reads them only once the quantizers have finished.
+    qp.queue = base == 0 ? tail.zero : nullptr;
+    qp.nqueue = base == 0 ? static_cast<int32_t>(tail.zero_ints) : 0;
+    for (int i = 0; i < cnt; ++i) {
+      qp.p[i].x = problems[base + i].X;
+      qp.p[i].xq = sl[base + i].first;
+      qp.p[i].xs = sl[base + i].second;
+      qp.p[i].k = problems[base + i].K;
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(cnt * M));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr = pdl_attr(true);
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_batched_kernel, qp);
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the batched activation quant kernel");
+  }
+  std::vector<int> small;
+  std::vector<MmaProblem> big;
+  std::vector<const int8_t*> big_xq;
+  for (int i = 0; i < count; ++i) {
+    const bitnet_i2s_problem& q = problems[i];
+    if (use_dp4a(M, q.K)) {
+      small.push_back(i);
+    } else {
+      big.push_back(make_mma_problem(q.packed, q.N, q.K, sl[i].second, q.Y, q.acc_or_null));
+      big_xq.push_back(sl[i].first);
+    }
+  }
+  bool first = true;
+  if (!small.empty()) {
+    const auto chunks = decode_chunks(
+        small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev);
+    for (size_t c = 0; c < chunks.size(); ++c) {
+      const size_t lo = chunks[c].first;
+      const size_t hi = chunks[c].second;
+      bp.count = static_cast<int32_t>(hi - lo);
+      bp.m = static_cast<int32_t>(M);
+      tail.assign(bp, c);
+      for (size_t i = lo; i < hi; ++i) {
+        const bitnet_i2s_problem& q = problems[small[i]];
+        bp.p[i - lo] = make_problem(q.packed, q.N, q.K, sl[small[i]].first, sl[small[i]].second,
+                                    q.Y, q.acc_or_null);
+      }
+      bitnet_status st = launch_dp4a(bp, s, /*pdl=*/true, dev, /*wait=*/first);
+      if (st != BITNET_OK) return st;
+      first = false;
+    }
+  }
+  if (!big.empty()) {
+    // run_mma_batches waits in its first launch only when asked to.
+    bitnet_status st = run_mma_batches(big, big_xq, M, /*pdl=*/true, s, dev, /*wait_first=*/first);
+    if (st != BITNET_OK) return st;
+  }
+  return BITNET_OK;
 }
 
 }  // namespace
@@ -570,8 +767,7 @@ bitnet_status bitnet_ternarize_absmean(const float* W, int64_t count, double eps
 
 size_t bitnet_i2s_quant_gemv_workspace_bytes(int64_t M, int64_t K) {
   if (M < 1 || K < 128 || K % 128 != 0) return 0;
-  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
-         align256(static_cast<size_t>(M) * sizeof(float));
+  return slot_bytes(M, K) + decode_tail_bytes(1, M);
 }
 
 bitnet_status bitnet_i2s_quant_gemv(const uint8_t* packed, int64_t N, int64_t K, const float* X,
@@ -591,23 +787,16 @@ bitnet_status bitnet_i2s_quant_gemv(const uint8_t* packed, int64_t N, int64_t K,
                 workspace_bytes, need);
   int dev;
   if ((st = check_device(&dev)) != BITNET_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int8_t* xq = static_cast<int8_t*>(workspace);
-  float* xs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                       align256(static_cast<size_t>(M) * static_cast<size_t>(K)));
-  // Quantize with PDL: the kernel waits for whatever precedes it, then lets
-  // the matmul launch so its weight loads overlap the quantization.
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(static_cast<unsigned>(M));
-  cfg.blockDim = dim3(256);
-  cfg.stream = s;
-  cudaLaunchAttribute attr = pdl_attr(true);
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, X, K, xq, xs);
-  if (e != cudaSuccess) return cuda_fail(e, "launch of the activation quant kernel");
-  st = run_matmul(packed, N, K, xq, xs, M, Y, acc_or_null, true, s, dev);
+  // One problem of the batched path: its workspace layout is the batched
+  // layout for one problem.
+  bitnet_i2s_problem q;
+  q.packed = packed;
+  q.N = N;
+  q.K = K;
+  q.X = X;
+  q.Y = Y;
+  q.acc_or_null = acc_or_null;
+  st = run_quant_batched(&q, 1, M, workspace, static_cast<cudaStream_t>(stream), dev);
   return st == BITNET_OK ? ok() : st;
 }
 
@@ -616,11 +805,11 @@ size_t bitnet_i2s_quant_gemv_batched_workspace_bytes(const bitnet_i2s_problem* p
   if (problems == nullptr || count < 1 || M < 1) return 0;
   size_t total = 0;
   for (int i = 0; i < count; ++i) {
-    const size_t one = bitnet_i2s_quant_gemv_workspace_bytes(M, problems[i].K);
-    if (one == 0) return 0;
-    total += one;
+    const int64_t k = problems[i].K;
+    if (k < 128 || k % 128 != 0) return 0;
+    total += slot_bytes(M, k);
   }
-  return total + queue_bytes(count);
+  return total + decode_tail_bytes(count, M);
 }
 
 bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, int count,
@@ -649,98 +838,14 @@ bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, 
   int dev;
   bitnet_status st = check_device(&dev);
   if (st != BITNET_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // 1. One launch quantizes every problem's tokens into the workspace.
-  // 2. Problems the integer-ALU decode kernel serves (M <= 2, K <= 8192) run
-  //    in launches of at most kMaxBatch problems, the rest in launches of at
-  //    most kMmaBatch problems on the tensor-core kernel.
-  // The first matmul launch waits for the quantizer; every later one is a
-  // dependent launch that skips the wait and starts streaming as soon as SMs
-  // free up: each launch in the chain starts only after every thread of the
-  // one before it has signalled, which the first launch's threads do only
-  // after their wait, so all of them start after the quantizer has finished;
-  // no matmul writes what another reads; and every CTA waits for the grid
-  // before its own before it exits, so the last launch completes last.
-  static thread_local QuantBatchParams qp;         // 32 KB: kept off the stack
-  static thread_local BatchParamsT<kMaxBatch> bp;  // 30 KB
-  std::vector<std::pair<int8_t*, float*>> sl(static_cast<size_t>(count));
-  int32_t* queue = nullptr;  // the decode launches' work counters, after the slots
-  {
-    uint8_t* w = static_cast<uint8_t*>(workspace);
-    for (int i = 0; i < count; ++i) {
-      sl[i] = {reinterpret_cast<int8_t*>(w),
-               reinterpret_cast<float*>(w + align256(static_cast<size_t>(M) * problems[i].K))};
-      w += bitnet_i2s_quant_gemv_workspace_bytes(M, problems[i].K);
-    }
-    queue = reinterpret_cast<int32_t*>(w);
-  }
-  for (int base = 0; base < count; base += kQuantBatch) {
-    const int cnt = std::min(kQuantBatch, count - base);
-    qp.count = cnt;
-    qp.m = static_cast<int32_t>(M);
-    // The first quantizer launch zeroes the counters; every decode launch
-    // reads its counter only once the quantizers have finished.
-    qp.queue = base == 0 ? queue : nullptr;
-    qp.nqueue = base == 0 ? static_cast<int32_t>(queue_bytes(count) / sizeof(int32_t)) : 0;
-    for (int i = 0; i < cnt; ++i) {
-      qp.p[i].x = problems[base + i].X;
-      qp.p[i].xq = sl[base + i].first;
-      qp.p[i].xs = sl[base + i].second;
-      qp.p[i].k = problems[base + i].K;
-    }
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(cnt * M));
-    cfg.blockDim = dim3(256);
-    cfg.stream = s;
-    cudaLaunchAttribute attr = pdl_attr(true);
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_batched_kernel, qp);
-    if (e != cudaSuccess) return cuda_fail(e, "launch of the batched activation quant kernel");
-  }
-  std::vector<int> small;
-  std::vector<MmaProblem> big;
-  std::vector<const int8_t*> big_xq;
-  for (int i = 0; i < count; ++i) {
-    const bitnet_i2s_problem& q = problems[i];
-    if (use_dp4a(M, q.K)) {
-      small.push_back(i);
-    } else {
-      big.push_back(make_mma_problem(q.packed, q.N, q.K, sl[i].second, q.Y, q.acc_or_null));
-      big_xq.push_back(sl[i].first);
-    }
-  }
-  bool first = true;
-  if (!small.empty()) {
-    const auto chunks = decode_chunks(
-        small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev);
-    for (size_t c = 0; c < chunks.size(); ++c) {
-      const size_t lo = chunks[c].first;
-      const size_t hi = chunks[c].second;
-      bp.count = static_cast<int32_t>(hi - lo);
-      bp.m = static_cast<int32_t>(M);
-      bp.queue = queue + c;
-      for (size_t i = lo; i < hi; ++i) {
-        const bitnet_i2s_problem& q = problems[small[i]];
-        bp.p[i - lo] = make_problem(q.packed, q.N, q.K, q.X, sl[small[i]].first,
-                                    sl[small[i]].second, q.Y, q.acc_or_null);
-      }
-      st = launch_dp4a(bp, s, /*pdl=*/true, dev, /*wait=*/first);
-      if (st != BITNET_OK) return st;
-      first = false;
-    }
-  }
-  if (!big.empty()) {
-    // run_mma_batches waits in its first launch only when asked to.
-    st = run_mma_batches(big, big_xq, M, /*pdl=*/true, s, dev, /*wait_first=*/first);
-    if (st != BITNET_OK) return st;
-  }
-  return ok();
+  st = run_quant_batched(problems, count, M, workspace, static_cast<cudaStream_t>(stream), dev);
+  return st == BITNET_OK ? ok() : st;
 }
 
 size_t bitnet_i2s_gemv_batched_workspace_bytes(int count) {
-  return count < 1 ? 0 : queue_bytes(count);
+  // The token count is not known here: the split area is sized for the
+  // decode kernel's largest, two tokens.
+  return count < 1 ? 0 : decode_tail_bytes(count, 2);
 }
 
 bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int count, int64_t M,
@@ -758,21 +863,20 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
   if (workspace != nullptr) {
     if (!aligned(workspace, 256))
       return fail(BITNET_ERR_ALIGN, "bitnet_i2s_gemv_batched: workspace must be 256-byte aligned");
-    if (workspace_bytes < queue_bytes(count))
+    if (workspace_bytes < bitnet_i2s_gemv_batched_workspace_bytes(count))
       return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_gemv_batched: workspace of %zu bytes < %zu",
-                  workspace_bytes, queue_bytes(count));
+                  workspace_bytes, bitnet_i2s_gemv_batched_workspace_bytes(count));
   }
   int dev;
   bitnet_status st = check_device(&dev);
   if (st != BITNET_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int32_t* queue = static_cast<int32_t*>(workspace);
   // Decode-kernel problems in launches of at most kMaxBatch, tensor-core
   // problems in launches of at most kMmaBatch.  The first launch is
-  // ordinary, or, with work counters, the one-warp grid that zeroes them
-  // after waiting for all earlier work on the stream; either way nothing
-  // later starts before that work has finished.  The later launches are
-  // dependent launches that start as SMs free up.
+  // ordinary, or, with a workspace, the grid that zeroes its counters after
+  // waiting for all earlier work on the stream; either way nothing later
+  // starts before that work has finished.  The later launches are dependent
+  // launches that start as SMs free up.
   static thread_local BatchParamsT<kMaxBatch> bp;
   std::vector<int> small;
   std::vector<MmaProblem> big;
@@ -786,24 +890,25 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
       big_xq.push_back(q.Xq);
     }
   }
+  const DecodeTail tail = decode_tail(workspace, count, 2);
   bool first = true;
   if (!small.empty()) {
     const auto chunks = decode_chunks(
         small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev);
     const size_t nchunks = chunks.size();
-    if (queue != nullptr) {
-      // A one-warp grid zeroes the counters once the work before this call is
-      // done; the first decode launch reads them after waiting for it.
+    if (workspace != nullptr) {
+      // One grid zeroes the counters once the work before this call is done;
+      // the first decode launch reads them after waiting for it.
       cudaLaunchConfig_t cfg;
       std::memset(&cfg, 0, sizeof(cfg));
       cfg.gridDim = dim3(1);
-      cfg.blockDim = dim3(32);
+      cfg.blockDim = dim3(256);
       cfg.stream = s;
       cudaLaunchAttribute attr = pdl_attr(true);
       cfg.attrs = &attr;
       cfg.numAttrs = 1;
-      cudaError_t e = cudaLaunchKernelEx(&cfg, zero_counters_kernel, queue,
-                                         static_cast<int32_t>(nchunks));
+      cudaError_t e = cudaLaunchKernelEx(&cfg, zero_counters_kernel, tail.zero,
+                                         static_cast<int32_t>(tail.zero_ints));
       if (e != cudaSuccess) return cuda_fail(e, "launch of the counter reset");
     }
     for (size_t c = 0; c < nchunks; ++c) {
@@ -811,12 +916,12 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
       const size_t hi = chunks[c].second;
       bp.count = static_cast<int32_t>(hi - lo);
       bp.m = static_cast<int32_t>(M);
-      bp.queue = queue != nullptr ? queue + c : nullptr;
+      tail.assign(bp, c);
       for (size_t i = lo; i < hi; ++i) {
         const bitnet_i2s_qproblem& q = problems[small[i]];
-        bp.p[i - lo] = make_problem(q.packed, q.N, q.K, nullptr, q.Xq, q.xs, q.Y, q.acc_or_null);
+        bp.p[i - lo] = make_problem(q.packed, q.N, q.K, q.Xq, q.xs, q.Y, q.acc_or_null);
       }
-      const bool after_reset = queue != nullptr && c == 0;
+      const bool after_reset = workspace != nullptr && c == 0;
       st = launch_dp4a(bp, s, /*pdl=*/!first || after_reset, dev, /*wait=*/after_reset);
       if (st != BITNET_OK) return st;
       first = false;
@@ -849,21 +954,50 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 
 namespace {
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device.  In host code the array's name is only a host-side stand-in, so
-// the address must come from the runtime; it is cached per device id.
+// cuCtxGetCurrent from the driver, without linking libcuda.
+PFN_cuCtxGetCurrent_v4000 ctx_fn() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  return fn;
+}
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address must come
+// from the runtime.  It is looked up once per device and context, with the
+// device current: a device reset destroys the context that held the library's
+// device image, and the next call sees a new context and looks the address up
+// again instead of using the old one.
 bitnet_status noalloc_scratch(int dev, void** out) {
+  struct Entry {
+    CUcontext ctx;
+    void* ptr;
+  };
   static std::mutex mu;
-  static void* cached[kMaxDevices];
+  static Entry cached[kMaxDevices];
+  CUcontext ctx = nullptr;
+  // The runtime call below makes the device's primary context current if no
+  // context is yet, so the context is read after it on a first call.
+  auto get_ctx = ctx_fn();
   std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
+  if (get_ctx != nullptr && get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  if (cached[dev].ptr == nullptr || ctx == nullptr || cached[dev].ctx != ctx) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
     if (p == nullptr) return fail(BITNET_ERR_CUDA, "static scratch has no device address");
-    cached[dev] = p;
+    if (get_ctx != nullptr && get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+    cached[dev].ptr = p;
+    cached[dev].ctx = ctx;  // null: unknown, looked up again on the next call
   }
-  *out = cached[dev];
+  *out = cached[dev].ptr;
   return BITNET_OK;
 }
 
@@ -893,6 +1027,141 @@ bitnet_status bitnet_i2s_quant_gemv_noalloc(const uint8_t* packed, int64_t N, in
   return bitnet_i2s_quant_gemv(packed, N, K, X, M, Y, acc_or_null, scratch,
                                kNoAllocScratchBytes, stream);
 }
+
+}  // extern "C"
+
+// ------------------------------------------------------ block-64 formats
+namespace {
+
+bitnet_status check_bn(const char* fn, const void* a, const void* b, int64_t N, int64_t K,
+                       bool r4) {
+  if (a == nullptr || b == nullptr) return fail(BITNET_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+  if (N < 1 || K < 64 || K % 64 != 0 || K > kMaxK || (r4 && N % 4 != 0))
+    return fail(BITNET_ERR_SHAPE, "%s: N=%lld, K=%lld (K a multiple of 64%s)", fn, (long long)N,
+                (long long)K, r4 ? ", N a multiple of 4" : "");
+  if (!aligned(a, 16) || !aligned(b, 16))
+    return fail(BITNET_ERR_ALIGN, "%s: buffers must be 16-byte aligned", fn);
+  return BITNET_OK;
+}
+
+int elementwise_grid(int64_t work, int dev) {
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256,
+                                                                 int64_t{sm_count(dev)} * 16)));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bitnet_iq2bn_bytes(int64_t N, int64_t K) {
+  if (N < 1 || K < 64 || K % 64 != 0) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) / 4 + 4 * static_cast<size_t>(N);
+}
+
+size_t bitnet_iq1bn_bytes(int64_t N, int64_t K) {
+  if (N < 1 || K < 64 || K % 64 != 0) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K / 64) * kIq1BnBlockBytes +
+         4 * static_cast<size_t>(N);
+}
+
+bitnet_status bitnet_iq2bn_pack(const float* W, int64_t N, int64_t K, int r4, uint8_t* out,
+                                void* stream) {
+  bitnet_status st = check_bn("bitnet_iq2bn_pack", W, out, N, K, r4 != 0);
+  if (st != BITNET_OK) return st;
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* d = reinterpret_cast<float*>(out + N * K / 4);
+  bn_row_absmax_kernel<<<static_cast<unsigned>(N), 256, 0, s>>>(W, K, d);
+  iq2bn_pack_kernel<<<elementwise_grid(N * K / 16, dev), 256, 0, s>>>(W, N, K, r4 != 0, out, d);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the IQ2_BN pack kernels");
+  return ok();
+}
+
+bitnet_status bitnet_iq2bn_dequant_f32(const uint8_t* packed, int64_t N, int64_t K, int r4,
+                                       float* W_out, void* stream) {
+  bitnet_status st = check_bn("bitnet_iq2bn_dequant_f32", packed, W_out, N, K, r4 != 0);
+  if (st != BITNET_OK) return st;
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  iq2bn_dequant_kernel<<<elementwise_grid(N * K / 16, dev), 256, 0,
+                         static_cast<cudaStream_t>(stream)>>>(
+      packed, N, K, r4 != 0, reinterpret_cast<const float*>(packed + N * K / 4), W_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the IQ2_BN dequantize kernel");
+  return ok();
+}
+
+bitnet_status bitnet_iq1bn_pack(const float* W, int64_t N, int64_t K, uint8_t* out, void* stream) {
+  bitnet_status st = check_bn("bitnet_iq1bn_pack", W, out, N, K, false);
+  if (st != BITNET_OK) return st;
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t code_bytes = N * (K / 64) * kIq1BnBlockBytes;
+  // The fp32 row scales follow the 13-byte blocks, so they are 4-byte
+  // aligned only when the number of blocks is a multiple of 4 (it is for
+  // every K of the BitNet shapes: K/64 = 40, 108, 128, 448).
+  if (code_bytes % 4 != 0)
+    return fail(BITNET_ERR_SHAPE, "bitnet_iq1bn_pack: N*(K/64) must be a multiple of 4");
+  float* d = reinterpret_cast<float*>(out + code_bytes);
+  bn_row_absmax_kernel<<<static_cast<unsigned>(N), 256, 0, s>>>(W, K, d);
+  iq1bn_pack_kernel<<<elementwise_grid(code_bytes, dev), 256, 0, s>>>(W, N, K, out, d);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the IQ1_BN pack kernels");
+  return ok();
+}
+
+bitnet_status bitnet_iq1bn_dequant_f32(const uint8_t* packed, int64_t N, int64_t K, float* W_out,
+                                       void* stream) {
+  bitnet_status st = check_bn("bitnet_iq1bn_dequant_f32", packed, W_out, N, K, false);
+  if (st != BITNET_OK) return st;
+  const int64_t code_bytes = N * (K / 64) * kIq1BnBlockBytes;
+  if (code_bytes % 4 != 0)
+    return fail(BITNET_ERR_SHAPE, "bitnet_iq1bn_dequant_f32: N*(K/64) must be a multiple of 4");
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  iq1bn_dequant_kernel<<<elementwise_grid(code_bytes, dev), 256, 0,
+                         static_cast<cudaStream_t>(stream)>>>(
+      packed, N, K, reinterpret_cast<const float*>(packed + code_bytes), W_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the IQ1_BN dequantize kernel");
+  return ok();
+}
+
+bitnet_status bitnet_iq2bn_r4_gemv(const uint8_t* packed, int64_t N, int64_t K, const int8_t* Xq,
+                                   const float* xs, int64_t M, float* Y, int32_t* acc_or_null,
+                                   void* stream) {
+  bitnet_status st = check_bn("bitnet_iq2bn_r4_gemv", packed, Xq, N, K, true);
+  if (st != BITNET_OK) return st;
+  if (xs == nullptr || Y == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_iq2bn_r4_gemv: null pointer argument");
+  if (M < 1 || M > 2 || K > kBnGemvMaxK || N > int64_t{0x7fffffff})
+    return fail(BITNET_ERR_SHAPE, "bitnet_iq2bn_r4_gemv: M=%lld (1..2), K=%lld (<= %d)",
+                (long long)M, (long long)K, kBnGemvMaxK);
+  if (!aligned(Y, 4) || !aligned(xs, 4) || (acc_or_null != nullptr && !aligned(acc_or_null, 4)))
+    return fail(BITNET_ERR_ALIGN, "bitnet_iq2bn_r4_gemv: Y, xs and acc must be 4-byte aligned");
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  const int64_t groups = N / 4;
+  const int grid = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>((groups + kBnGemvWarps - 1) / kBnGemvWarps, int64_t{sm_count(dev)} * 4)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 1)
+    iq2bn_r4_gemv_kernel<1><<<grid, kBnGemvWarps * 32, 0, s>>>(packed, N, K, Xq, xs, 1, Y,
+                                                               acc_or_null);
+  else
+    iq2bn_r4_gemv_kernel<2><<<grid, kBnGemvWarps * 32, 0, s>>>(packed, N, K, Xq, xs, 2, Y,
+                                                               acc_or_null);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the IQ2_BN_R4 matmul kernel");
+  return ok();
+}
+
+}  // extern "C"
+
+extern "C" {
 
 bitnet_status bitnet_debug_wait_timeout(int64_t timeout_ns, void* stream) {
   if (timeout_ns < 1000 || timeout_ns > 100000000)

@@ -63,16 +63,27 @@ constexpr int kGemvMaxK = 8192;      // the x slot holds M x K bytes, K <= 8192 
 constexpr int kGemvMaxKLong = 30720;  // ... or, in the one-token long-K variant, K <= 30720
 
 // One independent problem of a batch (device pointers and shape).
+//
+// Split K: a problem with few row tiles can have its K range cut into
+// `splits` slices of `cps` boxes each; a work item is then one (slice, row
+// tile) pair, numbered slice by slice.  Each item adds up its slice into
+// int32 partial sums in the workspace; the last of the slices of a row tile
+// to finish (per warp, counted in the workspace) adds the partials in slice
+// order and writes the outputs.  Integer sums are exact, so the results are
+// the same as without the split.
 struct BatchProblem {
   const uint8_t* packed;  // I2_S tensor [n, k]
-  const float* x;         // fp32 activations [m, k] (read by the batched quantizer)
   int8_t* xq;             // int8 activations [m, k]
   float* xs;              // per-token scales [m]
   float* y;               // [m, n]
   int32_t* acc;           // [m, n] or null
   int32_t n, k;
-  int32_t item_start;     // first global work item (row tile) of this problem
+  int32_t item_start;     // first global work item of this problem
   int32_t stage_start;    // first global stage (one box each) of this problem
+  int32_t splits;         // K slices (1: no split)
+  int32_t cps;            // boxes per slice (the last slice may have fewer)
+  int32_t part_off;       // partial sums: split_base + part_off, [tile][slice][MT][128]
+  int32_t cnt_off;        // arrival counters: cnt_base + cnt_off, [tile][4 warps]
 };
 
 template <int CAP>
@@ -85,7 +96,9 @@ struct BatchParamsT {
   int32_t dyn_start;     // items from here on are handed out through `queue`
   int32_t* queue;        // zeroed work counter, or null: every item in a fixed range
   int32_t static_stages; // stages of the items before dyn_start
-  int32_t pad[7];
+  int32_t pad;
+  int32_t* split_base;   // partial sums of split problems (workspace), or null
+  int32_t* cnt_base;     // their zeroed arrival counters (workspace), or null
   CUtensorMap tmap[CAP];  // per problem: packed bytes as [n rows, k/4 bytes], box 128 x 128
   BatchProblem p[CAP];
 };
@@ -132,8 +145,8 @@ __device__ __forceinline__ int find_problem_by_item(const BP& bp, int item) {
   return lo;
 }
 
-// First item whose first stage is at or after global stage `target`; items
-// of one problem all have ceil(k/512) stages.
+// First item whose first stage is at or after global stage `target`; the
+// items of one problem are counted as `cps` stages each.
 template <typename BP>
 __device__ __forceinline__ int first_item_at_stage(const BP& bp, int target) {
   if (target >= bp.total_stages) return bp.total_items;
@@ -144,10 +157,21 @@ __device__ __forceinline__ int first_item_at_stage(const BP& bp, int target) {
     else hi = mid - 1;
   }
   const BatchProblem& P = bp.p[lo];
-  const int nk = (P.k + 511) >> 9;
-  const int items = (P.n + kGemvTileRows - 1) / kGemvTileRows;
+  const int nk = P.cps;
+  const int items = ((P.n + kGemvTileRows - 1) / kGemvTileRows) * P.splits;
   const int off = (target - P.stage_start + nk - 1) / nk;
   return off >= items ? P.item_start + items : P.item_start + off;
+}
+
+// Row tile, slice and box range [kc_lo, kc_hi) of item `item` of problem P.
+__device__ __forceinline__ void split_item(const BatchProblem& P, int item, int* rt, int* sl,
+                                           int* kc_lo, int* kc_hi) {
+  const int tiles = (P.n + kGemvTileRows - 1) / kGemvTileRows;
+  const int local = item - P.item_start;
+  *sl = local / tiles;
+  *rt = local - *sl * tiles;
+  *kc_lo = *sl * P.cps;
+  *kc_hi = min((P.k + 511) >> 9, *kc_lo + P.cps);
 }
 
 template <int MT, int CAP, int KMAX = kGemvMaxK>
@@ -267,9 +291,10 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
         if (dyn && waited && !have_next && (!in_static || item + 1 >= item_hi)) grab();
         const int p = find_problem_by_item(bp, item);
         const BatchProblem& P = bp.p[p];
-        const int row0 = (item - P.item_start) * kGemvTileRows;
-        const int nk = (P.k + 511) >> 9;
-        for (int kc = 0; kc < nk; ++kc) {
+        int rt, sl, kc_lo, kc_hi;
+        split_item(P, item, &rt, &sl, &kc_lo, &kc_hi);
+        const int row0 = rt * kGemvTileRows;
+        for (int kc = kc_lo; kc < kc_hi; ++kc) {
           const int s = issued % S;
           if (issued >= S) {
             if (!waited) {
@@ -283,8 +308,8 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
               break;
             }
           }
-          int info = (kc == 0 ? 1 : 0) | (kc == nk - 1 ? 2 : 0);
-          if (kc == 0 && p != prev_p) {
+          int info = (kc == kc_lo ? 1 : 0) | (kc == kc_hi - 1 ? 2 : 0);
+          if (kc == kc_lo && p != prev_p) {
             // At most two switches wait for their activations: the slots.
             if (nsw - x_loaded >= 2) {
               if (!waited) wait_for_inputs();
@@ -374,7 +399,8 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
   float wscale = 0.0f;
   const uint8_t* xsm = xslots;
   int cur_slot = -1;
-  int k = 0, n = 0;
+  int k = 0, n = 0, splits = 1;
+  int kc_first = 0;  // first box of the current item
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     xsum[m] = 0;
@@ -412,12 +438,13 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
       xsm = xslots + slot * C::kXSlotBytes;
       k = bp.p[md.p].k;
       n = bp.p[md.p].n;
+      splits = bp.p[md.p].splits;
       wscale = xscal[4 * slot];
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         xsv[m] = xscal[4 * slot + 1 + m];
         int sum = 0;
-        if (m < m_tokens) {
+        if (m < m_tokens && splits == 1) {
           for (int off = lane * 16; off < k; off += 512) {
             const uint4 v = *reinterpret_cast<const uint4*>(xsm + m * k + off);
             sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
@@ -436,6 +463,26 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
         for (int m = 0; m < MT; ++m)
 #pragma unroll
           for (int g = 0; g < 4; ++g) a[i][m][g] = 0;
+      kc_first = md.kc;
+      if (splits > 1) {
+        // A slice of K: sum_k x over the slice's range only.
+        const int k_lo = md.kc * 512;
+        const int k_hi = min(k, k_lo + bp.p[md.p].cps * 512);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          int sum = 0;
+          if (m < m_tokens) {
+            for (int off = k_lo + lane * 16; off < k_hi; off += 512) {
+              const uint4 v = *reinterpret_cast<const uint4*>(xsm + m * k + off);
+              sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
+              sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
+              sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
+              sum = __dp4a(static_cast<int>(v.w), 0x01010101, sum);
+            }
+          }
+          xsum[m] = __reduce_add_sync(0xffffffffu, sum);
+        }
+      }
     }
     const int kblk = md.kc * 512 + 128 * cp;  // first weight of this lane's block
     if (kblk < k) {                            // blocks wholly past K are skipped
@@ -489,22 +536,69 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
       // Tile done: add the 4 block lanes of each row, then
       // y = ((float)acc * xs[m]) * s.
       const BatchProblem& P = bp.p[md.p];
+      if (splits == 1) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t row = static_cast<int64_t>(md.row0) + cw * 32 + rs + 8 * i;
+        for (int i = 0; i < 4; ++i) {
+          const int64_t row = static_cast<int64_t>(md.row0) + cw * 32 + rs + 8 * i;
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          int part = 0;
+          for (int m = 0; m < MT; ++m) {
+            int part = 0;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) part += a[i][m][j] >> gshift[j];
-          part += __shfl_xor_sync(0xffffffffu, part, 1);
-          part += __shfl_xor_sync(0xffffffffu, part, 2);
-          if (cp == 0 && m < m_tokens && row < n) {
-            const int dot = part - xsum[m];
-            P.y[m * static_cast<int64_t>(n) + row] =
-                __fmul_rn(__fmul_rn(__int2float_rn(dot), xsv[m]), wscale);
-            if (P.acc != nullptr) P.acc[m * static_cast<int64_t>(n) + row] = dot;
+            for (int j = 0; j < 4; ++j) part += a[i][m][j] >> gshift[j];
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            if (cp == 0 && m < m_tokens && row < n) {
+              const int dot = part - xsum[m];
+              P.y[m * static_cast<int64_t>(n) + row] =
+                  __fmul_rn(__fmul_rn(__int2float_rn(dot), xsv[m]), wscale);
+              if (P.acc != nullptr) P.acc[m * static_cast<int64_t>(n) + row] = dot;
+            }
           }
+        }
+      } else {
+        // One slice of a split problem: this warp's 32 rows of partial sums
+        // go to the workspace; the warp that brings the last slice of these
+        // rows adds all slices (in slice order) and writes the outputs.
+        const int rt = md.row0 / kGemvTileRows;
+        const int sl = kc_first / P.cps;
+        int32_t* tile_part =
+            bp.split_base + P.part_off + static_cast<int64_t>(rt) * splits * (MT * 128);
+        int32_t* mine = tile_part + static_cast<int64_t>(sl) * (MT * 128);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            int part = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) part += a[i][m][j] >> gshift[j];
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            if (cp == 0 && m < m_tokens) mine[m * 128 + cw * 32 + rs + 8 * i] = part - xsum[m];
+          }
+        }
+        __threadfence();
+        __syncwarp();
+        int32_t* cnt = bp.cnt_base + P.cnt_off + rt * 4 + cw;
+        int last = 0;
+        if (lane == 0) last = atomicAdd(cnt, 1) == splits - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          const int64_t row = static_cast<int64_t>(md.row0) + cw * 32 + lane;
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            if (m < m_tokens) {
+              int dot = 0;
+              for (int q = 0; q < splits; ++q)
+                dot += __ldcg(tile_part + q * (MT * 128) + m * 128 + cw * 32 + lane);
+              if (row < n) {
+                P.y[m * static_cast<int64_t>(n) + row] =
+                    __fmul_rn(__fmul_rn(__int2float_rn(dot), xsv[m]), wscale);
+                if (P.acc != nullptr) P.acc[m * static_cast<int64_t>(n) + row] = dot;
+              }
+            }
+          }
+          if (lane == 0) *cnt = 0;  // ready for the next call on this workspace
         }
       }
     }
@@ -513,7 +607,7 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
 
 // Zeroes the work counters of the decode launches that follow, once the
 // preceding grid (and with it every earlier user of the counters) is done.
-__global__ void __launch_bounds__(32) zero_counters_kernel(int32_t* queue, int32_t n) {
+__global__ void __launch_bounds__(256) zero_counters_kernel(int32_t* queue, int32_t n) {
   grid_dependency_wait();
   for (int i = threadIdx.x; i < n; i += blockDim.x) queue[i] = 0;
   grid_dependents_launch();

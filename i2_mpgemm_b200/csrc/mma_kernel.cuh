@@ -18,37 +18,42 @@
 // contiguous range of items balanced by their 512-wide K chunks, and streams
 // through it without stopping between items.
 //
-// Roles (320 threads):
-//   warp 0     TMA producer: per chunk one 128-row x 128-byte box of packed
-//              weights (512 k, four I2_S blocks) with the 128-byte swizzle,
-//              and one T x 128-byte box of Xq per I2_S block.
+// Roles (6 warps):
+//   warp 0     TMA producer.  Two rings: packed weights, one box of 128 rows
+//              x 128 bytes (a 512-wide K chunk, four I2_S blocks) per stage,
+//              and activations, a T x 128-byte box of Xq per I2_S block,
+//              kXB blocks per stage; both boxes use the 128-byte swizzle.
 //   warp 1     TMEM allocator and MMA issuer (one thread).
-//   warps 2-5  unpackers: thread r (= TMEM lane r) owns weight row r of the
-//              tile; per block it expands its row's 32 bytes into 4 groups x
-//              32 int8 values and stores them as 32 TMEM columns (one A
-//              slot).  In code mode they also add up each token's int8
-//              activations from the staged Xq boxes.
-//   warps 6-9  epilogue: y = ((float)acc * xs[m]) * s from the accumulator,
-//              token-major, while the next tile's MMAs run into the other
-//              accumulator buffer.
+//   warps 2-5  unpack and epilogue: thread r (= TMEM lane r) owns weight row
+//              r of the tile.  Per block it expands its row's 32 bytes into 4
+//              groups x 32 int8 values and stores them as 32 TMEM columns (one
+//              A slot); a weight stage is released as soon as its bytes are in
+//              registers.  At the end of an item the same warps read the
+//              accumulator of their lane quarter and write y = ((float)acc *
+//              xs[m]) * s, token-major.
+//
+// The MMA-issuing thread spends tens of cycles per small MMA, so a decode
+// tile keeps the tensor pipe fed only with several issuers per SM: small
+// token tiles run 3 or 4 CTAs per SM (TMEM 128 columns each), the
+// 128-token prefill tile 2.
 //
 // Unpack: the 32-bit word made of bytes 4i..4i+3 of a block, shifted right
 // by 6-2g and masked with 0x03030303, is the four codes of weights
 // 32g+4i .. 32g+4i+3 in byte order, i.e. one TMEM column of the A operand
 // for the MMA over k = 32g .. 32g+31.  Two variants:
 //   kCodes = true:  A holds the unsigned codes c = w+1 (two ALU ops per four
-//     weights); the epilogue subtracts sum_k x, which the unpackers add up
-//     from the Xq boxes on their way through shared memory.  For decode,
-//     where ALU issue is scarce and the MMAs are small.
+//     weights); the epilogue subtracts sum_k x, which the unpack warps add up
+//     from the activation boxes in shared memory.  For decode, where ALU
+//     issue is scarce and the MMAs are small.
 //   kCodes = false: A holds w itself (three more ALU ops per four weights).
 //     For prefill, where the unpack is amortised over 128 tokens.
 //
-// Pipelines: full/empty over the shared-memory stages (TMA -> unpack + MMA),
-// afull/aempty over four TMEM A slots handed over in pairs (unpack -> MMA),
-// dfull/dempty over two
-// accumulator buffers (MMA + unpackers -> epilogue -> MMA).  Every wait is
-// bounded (ptx.cuh); there are no named barriers, so a timed-out wait can
-// never leave another warp stuck.
+// Barriers: fullw/emptyw over the weight ring (TMA -> unpack), fullx/emptyx
+// over the activation ring (TMA -> MMA, and the unpack warps' token sums),
+// afull/aempty over the TMEM A slots (unpack -> MMA -> unpack), dfull/dempty
+// over the accumulator buffers (MMA -> epilogue -> MMA), xsum over the token
+// sums the unpack warps share.  Every wait is bounded (ptx.cuh); there are no
+// named barriers, so a timed-out wait can never leave another warp stuck.
 #pragma once
 
 #include "ptx.cuh"
@@ -87,23 +92,28 @@ struct MmaParamsT {
 
 template <int T, bool kCodes>
 struct MmaCfg {
-  static_assert(T % 16 == 0 && T >= 16 && T <= 128, "token tile");
-  static constexpr int kRows = 128;                     // MMA M
-  static constexpr int kThreads = 320;
-  static constexpr int kWTileBytes = kRows * 128;       // packed box: 128 rows x 128 B
-  static constexpr int kXBoxBytes = T * 128;            // Xq box: T rows x 128 B
-  static constexpr int kStageBytes = kWTileBytes + 4 * kXBoxBytes;
-  static constexpr int kStages = (T <= 16) ? 4 : (T <= 32 ? 3 : 2);
-  static constexpr int kCtasPerSm = (T <= 64) ? 2 : 1;
-  static constexpr int kASlots = 4;
-  static constexpr int kAGroup = 2;  // A slots handed over per handshake (two groups in flight)
-  static constexpr uint32_t kDCols = round32(T);        // one accumulator buffer
-  static constexpr uint32_t kACol = 2 * kDCols;         // A slots after both buffers
+  static_assert(T == 16 || T == 32 || T == 64 || T == 128, "token tile");
+  static constexpr int kRows = 128;  // MMA M
+  static constexpr int kThreads = 192;
+  static constexpr int kCtasPerSm = T <= 32 ? 4 : (T == 64 ? 3 : 2);
+  static constexpr int kDBufs = T <= 32 ? 2 : 1;        // accumulator buffers
+  static constexpr uint32_t kDCols = round32(T);        // columns of one buffer
+  static constexpr int kASlots = T <= 64 ? 2 : 4;       // 32-column A slots
+  static constexpr uint32_t kACol = kDBufs * kDCols;    // A slots after the buffers
   static constexpr uint32_t kTmemCols = pow2_at_least(kACol + 32u * kASlots);
-  static constexpr int kNumBars = 2 * kStages + 2 * kASlots + 4;
-  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes +
+  static constexpr int kWBytes = kRows * 128;           // weight box: 128 rows x 128 B
+  static constexpr int kWStages = 2;
+  static constexpr int kXBox = T * 128;                 // activation box: T rows x 128 B
+  static constexpr int kXB = T == 16 ? 4 : (T == 32 ? 2 : 1);  // blocks per activation stage
+  static constexpr int kXStageBytes = kXB * kXBox;
+  static constexpr int kXStages = T <= 32 ? 2 : 4;
+  static constexpr int kNumBars = 2 * kWStages + 2 * kXStages + 2 * kASlots + 2 * kDBufs + 2;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kWStages) * kWBytes +
+                                       static_cast<size_t>(kXStages) * kXStageBytes +
                                        kNumBars * 8 + 2 * T * 4 + 16;
   static constexpr uint32_t kIdesc = idesc_i8(128, T, !kCodes, true);
+  static_assert(kTmemCols * kCtasPerSm <= 512, "tensor memory per SM");
+  static_assert((kSmemBytes + 1024) * kCtasPerSm <= 228 * 1024, "shared memory per SM");
 };
 
 template <bool kCodes>
@@ -146,26 +156,28 @@ __device__ __forceinline__ int mma_first_item_at(const BP& bp, int target) {
 
 // Problem, row tile and token tile of an item.
 template <typename BP>
-__device__ __forceinline__ void mma_item(const BP& bp, int item, int T, int* p, int* rt, int* tt) {
+__device__ __forceinline__ void mma_item(const BP& bp, int item, int* p, int* rt, int* tt) {
   *p = mma_find_problem(bp, item);
   const MmaProblem& P = bp.p[*p];
   const int row_tiles = (P.n + 127) >> 7;
   const int local = item - P.item_start;
   *tt = local / row_tiles;
   *rt = local - *tt * row_tiles;
-  (void)T;
 }
 
 template <int T, bool kCodes, int CAP>
-__global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
+__global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
     i2s_mma_kernel(const __grid_constant__ MmaParamsT<CAP> bp) {
   using C = MmaCfg<T, kCodes>;
-  constexpr int S = C::kStages;
+  constexpr int WS = C::kWStages, XS = C::kXStages, AS = C::kASlots, DB = C::kDBufs;
+  constexpr int XB = C::kXB;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint8_t* wring = smem;
+  uint8_t* xring = smem + WS * C::kWBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xring + XS * C::kXStageBytes);
   int32_t* xsum_smem = reinterpret_cast<int32_t*>(bars + C::kNumBars);  // [2][T]
   uint32_t* misc = reinterpret_cast<uint32_t*>(xsum_smem + 2 * T);     // [0] tmem, [1] abort
   volatile uint32_t* abort_flag = misc + 1;
@@ -175,26 +187,35 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
   const int m_tokens = bp.m;
 
   const uint32_t bar0 = smem_u32(bars);
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-  auto afull_bar = [&](int t) { return bar0 + 8u * (2 * S + t); };
-  auto aempty_bar = [&](int t) { return bar0 + 8u * (2 * S + C::kASlots + t); };
-  auto dfull_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 * C::kASlots + b); };
-  auto dempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 * C::kASlots + 2 + b); };
+  auto fullw_bar = [&](int s) { return bar0 + 8u * s; };
+  auto emptyw_bar = [&](int s) { return bar0 + 8u * (WS + s); };
+  auto fullx_bar = [&](int s) { return bar0 + 8u * (2 * WS + s); };
+  auto emptyx_bar = [&](int s) { return bar0 + 8u * (2 * WS + XS + s); };
+  auto afull_bar = [&](int t) { return bar0 + 8u * (2 * WS + 2 * XS + t); };
+  auto aempty_bar = [&](int t) { return bar0 + 8u * (2 * WS + 2 * XS + AS + t); };
+  auto dfull_bar = [&](int b) { return bar0 + 8u * (2 * WS + 2 * XS + 2 * AS + b); };
+  auto dempty_bar = [&](int b) { return bar0 + 8u * (2 * WS + 2 * XS + 2 * AS + DB + b); };
+  auto xsum_bar = [&](int j) { return bar0 + 8u * (2 * WS + 2 * XS + 2 * AS + 2 * DB + j); };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 4 + 1);  // four unpack warps + one MMA commit
+    for (int s = 0; s < WS; ++s) {
+      mbar_init(fullw_bar(s), 1);
+      mbar_init(emptyw_bar(s), 4);  // the four unpack warps
     }
-    for (int t = 0; t < C::kASlots; ++t) {
+    for (int s = 0; s < XS; ++s) {
+      mbar_init(fullx_bar(s), 1);
+      mbar_init(emptyx_bar(s), kCodes ? 1 + 4 : 1);  // MMA commit (+ the token sums' reads)
+    }
+    for (int t = 0; t < AS; ++t) {
       mbar_init(afull_bar(t), 4);
       mbar_init(aempty_bar(t), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(dfull_bar(b), kCodes ? 1 + 4 : 1);  // MMA commit (+ the unpackers' sums)
-      mbar_init(dempty_bar(b), 4);                  // four epilogue warps
+    for (int b = 0; b < DB; ++b) {
+      mbar_init(dfull_bar(b), 1);
+      mbar_init(dempty_bar(b), 4);
     }
+    mbar_init(xsum_bar(0), 4);
+    mbar_init(xsum_bar(1), 4);
     misc[1] = 0u;
     fence_mbar_init();
   }
@@ -215,8 +236,6 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
   // once it has waited for this grid's inputs (at once when the launch reads
   // nothing the preceding grid writes); the producer does so after its own
   // lazy wait, and waits once more for the preceding grid before it exits.
-  // The stages every role consumes carry activations, which the producer
-  // requests only after its wait, so the other roles lose nothing by waiting.
   if (warp != 0 || lane != 0) {
     if (bp.pdl) grid_dependency_wait();
     grid_dependents_launch();
@@ -225,98 +244,102 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      // The weights of the first stages do not depend on the preceding grid:
-      // request them before waiting for it.  Each stage's barrier expects
-      // the weight and activation bytes together.
-      int issued = 0;
+      bool ok = true;
       bool waited = (bp.pdl == 0);
       if (waited) grid_dependents_launch();
-      bool ok = true;
-      int pre_item = item_lo, pre_kc = 0;  // chunk cursor of the activation loads
-      auto chunk_blocks = [&](const MmaProblem& P, int kc) { return min(4, (P.k >> 7) - 4 * kc); };
-      auto issue_x = [&](int s, int item, int kc) {
-        int p, rt, tt;
-        mma_item(bp, item, T, &p, &rt, &tt);
+      int wc = 0;  // weight stages issued
+      int xc = 0;  // activation stages issued
+      // The weights do not depend on the preceding grid: the first WS
+      // chunks' weights are requested before waiting for it, and their
+      // activations right after.
+      int pend_p[WS], pend_tt[WS], pend_kc[WS];
+      int npend = 0;
+      auto issue_x = [&](int p, int tt, int kc) -> bool {
         const MmaProblem& P = bp.p[p];
-        const int nb = chunk_blocks(P, kc);
-        uint8_t* st = smem + s * C::kStageBytes;
-        for (int q = 0; q < nb; ++q)
-          tma_load_2d(smem_u32(st + C::kWTileBytes + q * C::kXBoxBytes), &bp.tx[p],
-                      kc * 512 + q * 128, tt * T, full_bar(s));
+        const int nb = min(4, (P.k >> 7) - 4 * kc);
+        for (int q0 = 0; q0 < nb; q0 += XB, ++xc) {
+          const int s = xc % XS;
+          if (xc >= XS && !mbar_wait(emptyx_bar(s), ((xc / XS) - 1) & 1, abort_flag))
+            return false;
+          const int nbx = min(XB, nb - q0);
+          mbar_arrive_expect_tx(fullx_bar(s), nbx * C::kXBox);
+          uint8_t* dst = xring + s * C::kXStageBytes;
+          for (int q = 0; q < nbx; ++q)
+            tma_load_2d(smem_u32(dst + q * C::kXBox), &bp.tx[p], kc * 512 + (q0 + q) * 128,
+                        tt * T, fullx_bar(s));
+        }
+        return true;
       };
+      auto wait_inputs = [&]() -> bool {
+        grid_dependency_wait();
+        grid_dependents_launch();
+        waited = true;
+        for (int i = 0; i < npend; ++i)
+          if (!issue_x(pend_p[i], pend_tt[i], pend_kc[i])) return false;
+        npend = 0;
+        return true;
+      };
+      const uint64_t pol_w = l2_policy_evict_first();
       for (int item = item_lo; item < item_hi && ok; ++item) {
         int p, rt, tt;
-        mma_item(bp, item, T, &p, &rt, &tt);
+        mma_item(bp, item, &p, &rt, &tt);
         const MmaProblem& P = bp.p[p];
         prefetch_tensormap(&bp.tw[p]);
         prefetch_tensormap(&bp.tx[p]);
         const int nk = (P.k + 511) >> 9;
-        for (int kc = 0; kc < nk; ++kc) {
-          const int s = issued % S;
-          if (issued >= S) {
-            if (!waited) {
-              grid_dependency_wait();
-              grid_dependents_launch();
-              waited = true;
-              for (int i = 0; i < S; ++i) {  // activations of the stages issued so far
-                issue_x(i, pre_item, pre_kc);
-                int pp, r2, t2;
-                mma_item(bp, pre_item, T, &pp, &r2, &t2);
-                if (++pre_kc == ((bp.p[pp].k + 511) >> 9)) {
-                  pre_kc = 0;
-                  ++pre_item;
-                }
-              }
+        for (int kc = 0; kc < nk; ++kc, ++wc) {
+          const int s = wc % WS;
+          if (wc >= WS) {
+            if (!waited && !wait_inputs()) {
+              ok = false;
+              break;
             }
-            if (!mbar_wait(empty_bar(s), ((issued / S) - 1) & 1, abort_flag)) {
+            if (!mbar_wait(emptyw_bar(s), ((wc / WS) - 1) & 1, abort_flag)) {
               ok = false;
               break;
             }
           }
-          const int nb = chunk_blocks(P, kc);
-          mbar_arrive_expect_tx(full_bar(s), C::kWTileBytes + nb * C::kXBoxBytes);
-          tma_load_2d(smem_u32(smem + s * C::kStageBytes), &bp.tw[p], kc * 128, rt * 128,
-                      full_bar(s));
-          if (waited) issue_x(s, item, kc);
-          ++issued;
-        }
-      }
-      if (!waited && ok) {
-        grid_dependency_wait();
-        grid_dependents_launch();
-        waited = true;
-        for (int i = 0; i < issued; ++i) {
-          issue_x(i, pre_item, pre_kc);
-          int pp, r2, t2;
-          mma_item(bp, pre_item, T, &pp, &r2, &t2);
-          if (++pre_kc == ((bp.p[pp].k + 511) >> 9)) {
-            pre_kc = 0;
-            ++pre_item;
+          mbar_arrive_expect_tx(fullw_bar(s), C::kWBytes);
+          tma_load_2d_hint(smem_u32(wring + s * C::kWBytes), &bp.tw[p], kc * 128, rt * 128,
+                           fullw_bar(s), pol_w);
+          if (waited) {
+            if (!issue_x(p, tt, kc)) {
+              ok = false;
+              break;
+            }
+          } else {
+            pend_p[npend] = p;
+            pend_tt[npend] = tt;
+            pend_kc[npend] = kc;
+            ++npend;
           }
         }
       }
+      if (ok && !waited) ok = wait_inputs();
       // This CTA does not finish before the preceding grid has, so that the
       // completion of any grid in a chain implies that of all before it.
       grid_dependency_wait();
-      if (*abort_flag) {
+      if (*abort_flag || !ok) {
+        *abort_flag = 1u;
         // Let the copies already issued land before shared memory goes away
-        // (a stage whose activations were never requested cannot complete;
-        // its weight copy has landed by the end of this bounded wait).
-        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
-          mbar_wait(full_bar(i % S), (i / S) & 1, nullptr, kDrainTimeoutNs);
+        // (stages whose copies were never requested are not waited for).
+        for (int i = (wc > WS ? wc - WS : 0); i < wc; ++i)
+          mbar_wait(fullw_bar(i % WS), (i / WS) & 1, nullptr, kDrainTimeoutNs);
+        for (int i = (xc > XS ? xc - XS : 0); i < xc; ++i)
+          mbar_wait(fullx_bar(i % XS), (i / XS) & 1, nullptr, kDrainTimeoutNs);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = true;
-      int chunk = 0, blk = 0, ii = 0;
+      int blk = 0, xc = 0, ii = 0;
       for (int item = item_lo; item < item_hi && ok; ++item, ++ii) {
         int p, rt, tt;
-        mma_item(bp, item, T, &p, &rt, &tt);
+        mma_item(bp, item, &p, &rt, &tt);
         const MmaProblem& P = bp.p[p];
-        const int b = ii & 1;
-        if (ii >= 2 && !mbar_wait(dempty_bar(b), ((ii >> 1) - 1) & 1, abort_flag)) {
+        const int b = ii % DB;
+        if (ii >= DB && !mbar_wait(dempty_bar(b), ((ii / DB) - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -324,169 +347,178 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
         const uint32_t dcol = tmem + b * C::kDCols;
         const int nk = (P.k + 511) >> 9;
         bool first = true;
-        for (int kc = 0; kc < nk && ok; ++kc, ++chunk) {
-          const int s = chunk % S;
-          if (!mbar_wait(full_bar(s), (chunk / S) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
+        for (int kc = 0; kc < nk && ok; ++kc) {
           const int nb = min(4, (P.k >> 7) - 4 * kc);
-          const uint32_t xbase = smem_u32(smem + s * C::kStageBytes + C::kWTileBytes);
-          for (int bi = 0; bi < nb; ++bi, ++blk) {
-            const int t = blk & 3;
-            const int group = blk / C::kAGroup;
-            if (blk % C::kAGroup == 0) {
-              if (!mbar_wait(afull_bar(group & 1), (group >> 1) & 1, abort_flag)) {
+          for (int q0 = 0; q0 < nb && ok; q0 += XB, ++xc) {
+            const int s = xc % XS;
+            if (!mbar_wait(fullx_bar(s), (xc / XS) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const int nbx = min(XB, nb - q0);
+            const uint32_t xstage = smem_u32(xring + s * C::kXStageBytes);
+            for (int q = 0; q < nbx; ++q, ++blk) {
+              const int t = blk % AS;
+              if (!mbar_wait(afull_bar(t), (blk / AS) & 1, abort_flag)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-            }
-            const uint32_t xb = xbase + bi * C::kXBoxBytes;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              // K step g of this block: bytes 32g..32g+31 of each 128-byte Xq row.
-              mma_i8_tmem_a(dcol, tmem + C::kACol + 32u * t + 8u * g,
-                            smem_desc_sw128(xb + 32u * g), C::kIdesc, first ? 0u : 1u);
+              // K step g of this block: bytes 32g..32g+31 of each 128-byte Xq
+              // row, i.e. the descriptor's start address plus 2g (16-byte units).
+              const uint64_t bdesc = smem_desc_sw128(xstage + q * C::kXBox);
+              const uint32_t acol = tmem + C::kACol + 32u * t;
+              mma_i8_tmem_a(dcol, acol, bdesc, C::kIdesc, first ? 0u : 1u);
+              mma_i8_tmem_a(dcol, acol + 8u, bdesc + 2u, C::kIdesc, 1u);
+              mma_i8_tmem_a(dcol, acol + 16u, bdesc + 4u, C::kIdesc, 1u);
+              mma_i8_tmem_a(dcol, acol + 24u, bdesc + 6u, C::kIdesc, 1u);
               first = false;
+              tc_commit(aempty_bar(t));
             }
-            if (blk % C::kAGroup == C::kAGroup - 1) tc_commit(aempty_bar(group & 1));
+            if (ok) tc_commit(emptyx_bar(s));
           }
-          if (ok) tc_commit(empty_bar(s));
         }
         if (ok) tc_commit(dfull_bar(b));
       }
       // Our MMAs must be finished before TMEM is released.
       const int last = ii - 1;
       if (last >= 0)
-        mbar_wait(dfull_bar(last & 1), (last >> 1) & 1, nullptr,
+        mbar_wait(dfull_bar(last % DB), (last / DB) & 1, nullptr,
                   ok ? kWaitTimeoutNs : kDrainTimeoutNs);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ unpack
+  } else {
+    // ------------------------------------------------- unpack and epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const int ut = (warp - 2) * 32 + lane;  // 0..127 among the unpackers
+    const int ut = (warp - 2) * 32 + lane;  // 0..127 among the unpack warps
     bool ok = true;
-    int chunk = 0, blk = 0, ii = 0;
-    // A slots are handed over in pairs (C::kAGroup blocks): one store wait
-    // and one arrival per pair, and one commit per pair on the MMA side.
-    auto hand_over = [&](int group) {
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(afull_bar(group & 1));
-    };
+    int wc = 0, xc = 0, blk = 0, ii = 0;
     for (int item = item_lo; item < item_hi && ok; ++item, ++ii) {
       int p, rt, tt;
-      mma_item(bp, item, T, &p, &rt, &tt);
+      mma_item(bp, item, &p, &rt, &tt);
       const MmaProblem& P = bp.p[p];
       const int nk = (P.k + 511) >> 9;
-      int xacc[T / 16];  // code mode: token sums of this thread's Xq chunks
+      int xacc[T / 16];  // code mode: token sums over this thread's Xq chunks
 #pragma unroll
       for (int i = 0; i < T / 16; ++i) xacc[i] = 0;
-      for (int kc = 0; kc < nk && ok; ++kc, ++chunk) {
-        const int s = chunk % S;
-        ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (chunk / S) & 1, abort_flag));
+      for (int kc = 0; kc < nk && ok; ++kc, ++wc) {
+        const int s = wc % WS;
+        ok = __all_sync(0xffffffffu, mbar_wait(fullw_bar(s), (wc / WS) & 1, abort_flag));
         if (!ok) break;
         const int nb = min(4, (P.k >> 7) - 4 * kc);
-        const uint8_t* stage = smem + s * C::kStageBytes;
-        const uint8_t* wrow = stage + r * 128;
-        for (int bi = 0; bi < nb; ++bi, ++blk) {
-          const int t = blk & 3;
-          if (kCodes) {
-            // Token sums: the box holds T rows x 8 chunks of 16 bytes; this
-            // thread adds chunk (ut % 8) of rows ut / 8 + 16 i.  The swizzle
-            // only permutes chunks inside a row, so any chunk order will do.
-            const uint8_t* xb = stage + C::kWTileBytes + bi * C::kXBoxBytes;
+        // Row r of the weight box: its 128 bytes (four blocks) into registers,
+        // then the stage goes back to the producer.  The box was written with
+        // the 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r % 8).
+        const uint8_t* wrow = wring + s * C::kWBytes + r * 128;
+        uint4 wv4[8];
 #pragma unroll
-            for (int i = 0; i < T / 16; ++i) {
-              const uint4 v =
-                  *reinterpret_cast<const uint4*>(xb + (ut / 8 + 16 * i) * 128 + (ut % 8) * 16);
-              int a = xacc[i];
-              a = __dp4a(static_cast<int>(v.x), 0x01010101, a);
-              a = __dp4a(static_cast<int>(v.y), 0x01010101, a);
-              a = __dp4a(static_cast<int>(v.z), 0x01010101, a);
-              a = __dp4a(static_cast<int>(v.w), 0x01010101, a);
-              xacc[i] = a;
-            }
-          }
-          // The box was written with the 128-byte swizzle: 16-byte chunk c of
-          // row r sits at chunk c ^ (r % 8).
-          const uint4 c0 = *reinterpret_cast<const uint4*>(wrow + (((2 * bi) ^ (r & 7)) << 4));
-          const uint4 c1 = *reinterpret_cast<const uint4*>(wrow + (((2 * bi + 1) ^ (r & 7)) << 4));
-          const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          uint32_t a[32];
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) a[8 * g + i] = unpack_word<kCodes>(wv[i], g);
-          const int group = blk / C::kAGroup;
-          if (blk % C::kAGroup == 0 && group >= 2) {
-            // The pair of slots this group reuses has been read by its MMAs.
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(aempty_bar(group & 1), ((group >> 1) - 1) & 1, abort_flag));
-            if (!ok) break;
-          }
-          tc_fence_after();
-          tmem_st_32x32b_x32(tmem + lane_base + C::kACol + 32u * t, a);
-          if (blk % C::kAGroup == C::kAGroup - 1) hand_over(group);
-        }
+        for (int c = 0; c < 8; ++c)
+          wv4[c] = *reinterpret_cast<const uint4*>(wrow + ((c ^ (r & 7)) << 4));
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive(empty_bar(s));
+        if (lane == 0) mbar_arrive(emptyw_bar(s));
+        for (int q0 = 0; q0 < nb && ok; q0 += XB, ++xc) {
+          const int xs_ = xc % XS;
+          const int nbx = min(XB, nb - q0);
+          if (kCodes) {
+            // Token sums: each activation box holds T rows x 8 chunks of 16
+            // bytes; this thread adds chunk (ut % 8) of rows ut / 8 + 16 i.
+            // The swizzle only permutes chunks inside a row, so any chunk
+            // order will do.
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(fullx_bar(xs_), (xc / XS) & 1, abort_flag));
+            if (!ok) break;
+            const uint8_t* xst = xring + xs_ * C::kXStageBytes;
+            for (int q = 0; q < nbx; ++q) {
+#pragma unroll
+              for (int i = 0; i < T / 16; ++i) {
+                const uint4 v = *reinterpret_cast<const uint4*>(
+                    xst + q * C::kXBox + (ut / 8 + 16 * i) * 128 + (ut % 8) * 16);
+                int a = xacc[i];
+                a = __dp4a(static_cast<int>(v.x), 0x01010101, a);
+                a = __dp4a(static_cast<int>(v.y), 0x01010101, a);
+                a = __dp4a(static_cast<int>(v.z), 0x01010101, a);
+                a = __dp4a(static_cast<int>(v.w), 0x01010101, a);
+                xacc[i] = a;
+              }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(emptyx_bar(xs_));
+          }
+          for (int q = 0; q < nbx; ++q, ++blk) {
+            const int bi = q0 + q;  // block of the weight stage
+            const uint4 c0 = wv4[2 * bi], c1 = wv4[2 * bi + 1];
+            const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            uint32_t a[32];
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) a[8 * g + i] = unpack_word<kCodes>(wv[i], g);
+            const int t = blk % AS;
+            if (blk >= AS) {
+              // The slot's previous block has been read by its MMAs.
+              ok = __all_sync(0xffffffffu,
+                              mbar_wait(aempty_bar(t), ((blk / AS) - 1) & 1, abort_flag));
+              if (!ok) break;
+            }
+            tc_fence_after();
+            tmem_st_32x32b_x32(tmem + lane_base + C::kACol + 32u * t, a);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(afull_bar(t));
+          }
+        }
       }
-      if (kCodes && ok) {
-        // Sum the 8 chunk threads of each row, publish with the dfull arrival.
-        const int b = ii & 1;
-        if (ii >= 2)
-          ok = __all_sync(0xffffffffu, mbar_wait(dempty_bar(b), ((ii >> 1) - 1) & 1, abort_flag));
-        if (!ok) break;
+      if (!ok) break;
+      // ---- epilogue of this item
+      const int b = ii % DB;
+      if (kCodes) {
+        // Sum the 8 chunk threads of each token; share through shared memory.
 #pragma unroll
         for (int i = 0; i < T / 16; ++i) {
           int v = xacc[i];
           v += __shfl_xor_sync(0xffffffffu, v, 1);
           v += __shfl_xor_sync(0xffffffffu, v, 2);
           v += __shfl_xor_sync(0xffffffffu, v, 4);
-          if ((ut & 7) == 0) xsum_smem[b * T + ut / 8 + 16 * i] = v;
+          if ((ut & 7) == 0) xsum_smem[(ii & 1) * T + ut / 8 + 16 * i] = v;
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(dfull_bar(b));
+        if (lane == 0) mbar_arrive(xsum_bar(ii & 1));
       }
-    }
-    if (ok && blk % C::kAGroup != 0) hand_over(blk / C::kAGroup);  // a last, partial pair
-    tmem_st_wait();  // no store of this thread outlives it
-  } else {
-    // ---------------------------------------------------------- epilogue
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    int ii = 0;
-    for (int item = item_lo; item < item_hi; ++item, ++ii) {
-      int p, rt, tt;
-      mma_item(bp, item, T, &p, &rt, &tt);
-      const MmaProblem& P = bp.p[p];
-      const int b = ii & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(dfull_bar(b), (ii >> 1) & 1, abort_flag))) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(dfull_bar(b), (ii / DB) & 1, abort_flag));
+      if (!ok) break;
+      if (kCodes) {
+        ok = __all_sync(0xffffffffu, mbar_wait(xsum_bar(ii & 1), (ii >> 1) & 1, abort_flag));
+        if (!ok) break;
+      }
       tc_fence_after();
       const float s = *reinterpret_cast<const float*>(P.packed + static_cast<int64_t>(P.n) * (P.k >> 2));
       const int64_t n = static_cast<int64_t>(rt) * 128 + r;
       const int64_t tok0 = static_cast<int64_t>(tt) * T;
+      const int64_t nn = P.n;
+      float* __restrict__ yb = P.y;
+      int32_t* __restrict__ ab = P.acc;
+      const float* __restrict__ xsb = P.xs;
 #pragma unroll 1
       for (int c0 = 0; c0 < T; c0 += 16) {
         if (tok0 + c0 >= m_tokens) break;  // warp-uniform
+        float xsv[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          xsv[j] = (tok0 + c0 + j < m_tokens) ? __ldg(xsb + tok0 + c0 + j) : 0.0f;
         uint32_t v[16];
         tmem_ld_32x32b_x16(tmem + lane_base + b * C::kDCols + c0, v);
         tmem_ld_wait();
-        if (n < P.n) {
+        if (n < nn) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int64_t tok = tok0 + c0 + j;
             if (tok < m_tokens) {
               int32_t a = static_cast<int32_t>(v[j]);
-              if (kCodes) a -= xsum_smem[b * T + c0 + j];
-              P.y[tok * P.n + n] = __fmul_rn(__fmul_rn(__int2float_rn(a), __ldg(P.xs + tok)), s);
-              if (P.acc != nullptr) P.acc[tok * P.n + n] = a;
+              if (kCodes) a -= xsum_smem[(ii & 1) * T + c0 + j];
+              yb[tok * nn + n] = __fmul_rn(__fmul_rn(__int2float_rn(a), xsv[j]), s);
+              if (ab != nullptr) ab[tok * nn + n] = a;
             }
           }
         }
@@ -495,6 +527,7 @@ __global__ void __launch_bounds__(320, MmaCfg<T, kCodes>::kCtasPerSm)
       __syncwarp();
       if (lane == 0) mbar_arrive(dempty_bar(b));
     }
+    tmem_st_wait();  // no store of this thread outlives it
   }
 
   tc_fence_before();

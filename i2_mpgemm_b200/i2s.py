@@ -46,6 +46,13 @@ SIGNATURES = {
     "bitnet_i2s_gemv_batched_workspace_bytes": (_SZ, [_I32]),
     "bitnet_i2s_gemv_batched": (_I32, [_VP, _I32, _I64, _VP, _SZ, _VP]),
     "bitnet_i2s_quant_gemv_noalloc": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP]),
+    "bitnet_iq2bn_bytes": (_SZ, [_I64, _I64]),
+    "bitnet_iq1bn_bytes": (_SZ, [_I64, _I64]),
+    "bitnet_iq2bn_pack": (_I32, [_VP, _I64, _I64, _I32, _VP, _VP]),
+    "bitnet_iq2bn_dequant_f32": (_I32, [_VP, _I64, _I64, _I32, _VP, _VP]),
+    "bitnet_iq1bn_pack": (_I32, [_VP, _I64, _I64, _VP, _VP]),
+    "bitnet_iq1bn_dequant_f32": (_I32, [_VP, _I64, _I64, _VP, _VP]),
+    "bitnet_iq2bn_r4_gemv": (_I32, [_VP, _I64, _I64, _VP, _VP, _I64, _VP, _VP, _VP]),
     "bitnet_debug_wait_timeout": (_I32, [_I64, _VP]),
     "bitnet_device_status": (_I32, []),
     "bitnet_last_error": (ctypes.c_char_p, []),
@@ -78,9 +85,22 @@ def _check(status: int) -> None:
         raise BitnetError(status, lib.bitnet_last_error().decode(errors="replace"))
 
 
-def _stream(stream) -> int | None:
-    s = torch.cuda.current_stream() if stream is None else stream
-    return s.cuda_stream or None
+def _run(dev: torch.device, fn, *args, stream=None) -> None:
+    """Call C entry point `fn(*args, stream)` with `dev` as the current CUDA
+    device, on `stream` or, by default, the current torch stream of `dev`.
+    The library works on whichever device is current, so a call on tensors of
+    another device must switch to theirs first."""
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        if s.device != dev:
+            raise ValueError(f"stream is on {s.device}, the tensors on {dev}")
+        _check(fn(*args, s.cuda_stream or None))
+
+
+def _same_device(dev: torch.device, **tensors) -> None:
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -112,7 +132,8 @@ def bitnet_i2s_pack(w: torch.Tensor, packed: torch.Tensor | None = None, stream=
     if packed is None:
         packed = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=w.device)
     _need(packed, "packed", torch.uint8, nbytes)
-    _check(lib.bitnet_i2s_pack(_ptr(w), n, k, _ptr(packed), _stream(stream)))
+    _same_device(w.device, packed=packed)
+    _run(w.device, lib.bitnet_i2s_pack, _ptr(w), n, k, _ptr(packed), stream=stream)
     return packed
 
 
@@ -125,7 +146,8 @@ def bitnet_act_quant_i8(x: torch.Tensor, xq: torch.Tensor | None = None,
     xs = torch.empty(m, dtype=torch.float32, device=x.device) if xs is None else xs
     _need(xq, "Xq", torch.int8, m * k)
     _need(xs, "xs", torch.float32, m)
-    _check(lib.bitnet_act_quant_i8(_ptr(x), m, k, _ptr(xq), _ptr(xs), _stream(stream)))
+    _same_device(x.device, Xq=xq, xs=xs)
+    _run(x.device, lib.bitnet_act_quant_i8, _ptr(x), m, k, _ptr(xq), _ptr(xs), stream=stream)
     return xq, xs
 
 
@@ -142,7 +164,8 @@ def _matmul(fn, packed, n, k, xq, xs, y, acc, want_acc, stream):
         acc = torch.empty((m, n), dtype=torch.int32, device=dev)
     if acc is not None:
         _need(acc, "acc", torch.int32, m * n)
-    _check(fn(_ptr(packed), n, k, _ptr(xq), _ptr(xs), m, _ptr(y), _ptr(acc), _stream(stream)))
+    _same_device(dev, Xq=xq, xs=xs, Y=y, acc=acc)
+    _run(dev, fn, _ptr(packed), n, k, _ptr(xq), _ptr(xs), m, _ptr(y), _ptr(acc), stream=stream)
     return (y, acc) if acc is not None else y
 
 
@@ -161,7 +184,8 @@ def bitnet_i2s_dequant_f32(packed, n, k, w_out=None, stream=None):
     _need(packed, "packed", torch.uint8, bitnet_i2s_packed_bytes(n, k))
     w_out = torch.empty((n, k), dtype=torch.float32, device=packed.device) if w_out is None else w_out
     _need(w_out, "W_out", torch.float32, n * k)
-    _check(lib.bitnet_i2s_dequant_f32(_ptr(packed), n, k, _ptr(w_out), _stream(stream)))
+    _same_device(packed.device, W_out=w_out)
+    _run(packed.device, lib.bitnet_i2s_dequant_f32, _ptr(packed), n, k, _ptr(w_out), stream=stream)
     return w_out
 
 
@@ -173,8 +197,9 @@ def bitnet_ternarize_absmean(w, eps: float = 1e-5, w_out=None, stream=None):
     gamma = torch.empty(1, dtype=torch.float64, device=w.device)
     ws = torch.empty(int(lib.bitnet_ternarize_absmean_workspace_bytes()), dtype=torch.uint8,
                      device=w.device)
-    _check(lib.bitnet_ternarize_absmean(_ptr(w), w.numel(), float(eps), _ptr(w_out), _ptr(gamma),
-                                        _ptr(ws), ws.numel(), _stream(stream)))
+    _same_device(w.device, W_out=w_out)
+    _run(w.device, lib.bitnet_ternarize_absmean, _ptr(w), w.numel(), float(eps), _ptr(w_out),
+         _ptr(gamma), _ptr(ws), ws.numel(), stream=stream)
     return w_out, gamma
 
 
@@ -204,8 +229,9 @@ def bitnet_i2s_quant_gemv(packed, n, k, x, y=None, acc=None, workspace=None, wan
         acc = torch.empty((m, n), dtype=torch.int32, device=dev)
     if acc is not None:
         _need(acc, "acc", torch.int32, m * n)
-    _check(lib.bitnet_i2s_quant_gemv(_ptr(packed), n, k, _ptr(x), m, _ptr(y), _ptr(acc),
-                                     _ptr(workspace), workspace.numel(), _stream(stream)))
+    _same_device(dev, X=x, Y=y, acc=acc, workspace=workspace)
+    _run(dev, lib.bitnet_i2s_quant_gemv, _ptr(packed), n, k, _ptr(x), m, _ptr(y), _ptr(acc),
+         _ptr(workspace), workspace.numel(), stream=stream)
     return (y, acc) if acc is not None else y
 
 
@@ -245,12 +271,14 @@ class BatchedQuantGemv:
             dev = problems[0][0].device
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         _need(workspace, "workspace", torch.uint8, need)
+        self.device = problems[0][0].device
+        for t in self.tensors + [workspace]:
+            _same_device(self.device, tensor=t)
         self.workspace = workspace
 
     def run(self, stream=None) -> None:
-        _check(lib.bitnet_i2s_quant_gemv_batched(self.array, self.count, self.m,
-                                                 self.workspace.data_ptr(),
-                                                 self.workspace.numel(), _stream(stream)))
+        _run(self.device, lib.bitnet_i2s_quant_gemv_batched, self.array, self.count, self.m,
+             self.workspace.data_ptr(), self.workspace.numel(), stream=stream)
 
 
 def bitnet_i2s_quant_gemv_batched(problems, m: int, workspace=None, stream=None) -> None:
@@ -293,13 +321,16 @@ class BatchedGemv:
             workspace = torch.empty(need, dtype=torch.uint8, device=problems[0][0].device)
         if workspace is not None:
             _need(workspace, "workspace", torch.uint8)
+        self.device = problems[0][0].device
+        for t in self.tensors + [workspace]:
+            _same_device(self.device, tensor=t)
         self.workspace = workspace
 
     def run(self, stream=None) -> None:
         ws = self.workspace
-        _check(lib.bitnet_i2s_gemv_batched(self.array, self.count, self.m,
-                                           None if ws is None else ws.data_ptr(),
-                                           0 if ws is None else ws.numel(), _stream(stream)))
+        _run(self.device, lib.bitnet_i2s_gemv_batched, self.array, self.count, self.m,
+             None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
+             stream=stream)
 
 
 def bitnet_i2s_gemv_batched(problems, m: int, workspace=True, stream=None) -> None:
@@ -321,8 +352,83 @@ def bitnet_i2s_quant_gemv_noalloc(packed, n, k, x, y=None, acc=None, want_acc=Fa
         acc = torch.empty((m, n), dtype=torch.int32, device=dev)
     if acc is not None:
         _need(acc, "acc", torch.int32, m * n)
-    _check(lib.bitnet_i2s_quant_gemv_noalloc(_ptr(packed), n, k, _ptr(x), m, _ptr(y), _ptr(acc),
-                                             _stream(stream)))
+    # The static scratch is chosen by the current device: the call runs with
+    # the tensors' device current.
+    _same_device(dev, X=x, Y=y, acc=acc)
+    _run(dev, lib.bitnet_i2s_quant_gemv_noalloc, _ptr(packed), n, k, _ptr(x), m, _ptr(y),
+         _ptr(acc), stream=stream)
+    return (y, acc) if acc is not None else y
+
+
+def bitnet_iq2bn_bytes(n: int, k: int) -> int:
+    return int(lib.bitnet_iq2bn_bytes(n, k))
+
+
+def bitnet_iq1bn_bytes(n: int, k: int) -> int:
+    return int(lib.bitnet_iq1bn_bytes(n, k))
+
+
+def bitnet_iq2bn_pack(w: torch.Tensor, r4: bool = False, out=None, stream=None):
+    """fp32 W[N,K] -> uint8 IQ2_BN (or IQ2_BN_R4) tensor."""
+    _need(w, "W", torch.float32)
+    n, k = w.shape
+    nbytes = bitnet_iq2bn_bytes(n, k)
+    out = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=w.device) if out is None else out
+    _need(out, "out", torch.uint8, nbytes)
+    _same_device(w.device, out=out)
+    _run(w.device, lib.bitnet_iq2bn_pack, _ptr(w), n, k, int(bool(r4)), _ptr(out), stream=stream)
+    return out
+
+
+def bitnet_iq2bn_dequant_f32(packed, n, k, r4: bool = False, w_out=None, stream=None):
+    _need(packed, "packed", torch.uint8, bitnet_iq2bn_bytes(n, k))
+    w_out = torch.empty((n, k), dtype=torch.float32, device=packed.device) if w_out is None else w_out
+    _need(w_out, "W_out", torch.float32, n * k)
+    _same_device(packed.device, W_out=w_out)
+    _run(packed.device, lib.bitnet_iq2bn_dequant_f32, _ptr(packed), n, k, int(bool(r4)),
+         _ptr(w_out), stream=stream)
+    return w_out
+
+
+def bitnet_iq1bn_pack(w: torch.Tensor, out=None, stream=None):
+    """fp32 W[N,K] -> uint8 IQ1_BN tensor."""
+    _need(w, "W", torch.float32)
+    n, k = w.shape
+    nbytes = bitnet_iq1bn_bytes(n, k)
+    out = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=w.device) if out is None else out
+    _need(out, "out", torch.uint8, nbytes)
+    _same_device(w.device, out=out)
+    _run(w.device, lib.bitnet_iq1bn_pack, _ptr(w), n, k, _ptr(out), stream=stream)
+    return out
+
+
+def bitnet_iq1bn_dequant_f32(packed, n, k, w_out=None, stream=None):
+    _need(packed, "packed", torch.uint8, bitnet_iq1bn_bytes(n, k))
+    w_out = torch.empty((n, k), dtype=torch.float32, device=packed.device) if w_out is None else w_out
+    _need(w_out, "W_out", torch.float32, n * k)
+    _same_device(packed.device, W_out=w_out)
+    _run(packed.device, lib.bitnet_iq1bn_dequant_f32, _ptr(packed), n, k, _ptr(w_out),
+         stream=stream)
+    return w_out
+
+
+def bitnet_iq2bn_r4_gemv(packed, n, k, xq, xs, y=None, acc=None, want_acc=False, stream=None):
+    """Decode matmul (M = Xq.shape[0] in 1..2) on an IQ2_BN_R4 tensor."""
+    _need(packed, "packed", torch.uint8, bitnet_iq2bn_bytes(n, k))
+    _need(xq, "Xq", torch.int8)
+    m = xq.shape[0]
+    _need(xq, "Xq", torch.int8, m * k)
+    _need(xs, "xs", torch.float32, m)
+    dev = packed.device
+    y = torch.empty((m, n), dtype=torch.float32, device=dev) if y is None else y
+    _need(y, "Y", torch.float32, m * n)
+    if want_acc and acc is None:
+        acc = torch.empty((m, n), dtype=torch.int32, device=dev)
+    if acc is not None:
+        _need(acc, "acc", torch.int32, m * n)
+    _same_device(dev, Xq=xq, xs=xs, Y=y, acc=acc)
+    _run(dev, lib.bitnet_iq2bn_r4_gemv, _ptr(packed), n, k, _ptr(xq), _ptr(xs), m, _ptr(y),
+         _ptr(acc), stream=stream)
     return (y, acc) if acc is not None else y
 
 
@@ -333,7 +439,8 @@ def bitnet_device_status() -> None:
 
 def bitnet_debug_wait_timeout(timeout_ns: int = 1_000_000, stream=None) -> None:
     """Launch one device wait that runs out after timeout_ns (failure-detection check)."""
-    _check(lib.bitnet_debug_wait_timeout(int(timeout_ns), _stream(stream)))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _run(dev, lib.bitnet_debug_wait_timeout, int(timeout_ns), stream=stream)
 
 
 def bitnet_last_error() -> str:

@@ -144,7 +144,9 @@ BITNET_API bitnet_status bitnet_ternarize_absmean(const float* W, int64_t count,
                                                   size_t workspace_bytes, void* stream);
 
 /* Bytes of device scratch that bitnet_i2s_quant_gemv needs for M tokens of
- * length K (the int8 activations and their scales).  0 for a bad shape. */
+ * length K: the int8 activations and their scales and, for one or two
+ * tokens, room for split-K partial sums (256 KB per token) and their
+ * counters.  0 for a bad shape. */
 BITNET_API size_t bitnet_i2s_quant_gemv_workspace_bytes(int64_t M, int64_t K);
 
 /* Activation quantization followed by the ternary matmul: exactly
@@ -154,7 +156,13 @@ BITNET_API size_t bitnet_i2s_quant_gemv_workspace_bytes(int64_t M, int64_t K);
  *   workspace: caller-owned device scratch of at least
  *     bitnet_i2s_quant_gemv_workspace_bytes(M,K) bytes, 256-byte aligned;
  *     it must not be used by other work that may run at the same time.
- *   Other arguments as bitnet_i2s_gemv; M >= 1. */
+ *     Its contents need not be initialised: the call zeroes what it counts.
+ *   With one or two tokens and fewer 128-row tiles than the GPU runs CTAs of
+ *   the decode kernel at once, the call cuts K into slices that run on
+ *   separate SMs and adds their int32 partial sums in the workspace; integer
+ *   sums are exact, so the results are those of the unsplit contraction.
+ *   Other arguments as bitnet_i2s_gemv; M >= 1.  The same as
+ *   bitnet_i2s_quant_gemv_batched with one problem. */
 BITNET_API bitnet_status bitnet_i2s_quant_gemv(const uint8_t* packed, int64_t N, int64_t K, const float* X,
                                     int64_t M, float* Y, int32_t* acc_or_null, void* workspace,
                                     size_t workspace_bytes, void* stream);
@@ -188,7 +196,12 @@ BITNET_API size_t bitnet_i2s_quant_gemv_batched_workspace_bytes(const bitnet_i2s
  *   problems: HOST array of `count` descriptors, read during the call only.
  *   workspace: device scratch of at least
  *     bitnet_i2s_quant_gemv_batched_workspace_bytes(problems, count, M) bytes,
- *     256-byte aligned, not shared with work that may run at the same time.
+ *     256-byte aligned, not shared with work that may run at the same time;
+ *     its contents need not be initialised.
+ * When a decode launch has fewer 128-row tiles than it runs CTAs (a few
+ * small projections, or one of them), each problem's K is cut into slices of
+ * whole 512-weight boxes that run on separate SMs; the slices' int32 partial
+ * sums meet in the workspace and the last slice of each tile adds them.
  * The problems' outputs must not overlap each other or any input. */
 BITNET_API bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem* problems, int count,
                                                        int64_t M, void* workspace,
@@ -219,9 +232,10 @@ BITNET_API size_t bitnet_i2s_gemv_batched_workspace_bytes(int count);
  *     bitnet_i2s_gemv_batched_workspace_bytes(count) bytes, 256-byte aligned,
  *     not shared with work that may run at the same time.  With it, the
  *     integer-ALU launches hand out their tiles through work counters there
- *     (zeroed on `stream` first), which evens out the SMs' finishing times;
- *     without it each CTA takes a fixed range of tiles.  Results are the same
- *     either way. */
+ *     (zeroed on `stream` first), which evens out the SMs' finishing times,
+ *     and split K as bitnet_i2s_quant_gemv_batched does when a launch has
+ *     few row tiles; without it each CTA takes a fixed range of whole tiles.
+ *     Results are the same either way. */
 BITNET_API bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int count,
                                                  int64_t M, void* workspace,
                                                  size_t workspace_bytes, void* stream);
@@ -238,8 +252,16 @@ BITNET_API bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* prob
  *     BITNET_ERR_SHAPE before anything is launched.
  *   - It allocates nothing (no cudaMalloc, cudaFree or allocating library
  *     routine).  The first call on a device looks the array's address up
- *     once for that device (with the device current); make that first call
- *     before any stream capture.
+ *     for that device and its current context (with the device current) and
+ *     keeps it; a call that finds a different current context on the device
+ *     (after a device reset, say) looks it up again.  Make the first call on
+ *     each device before any stream capture.
+ *   - That first lookup can load the library's device image onto the device
+ *     (CUDA loads modules lazily by default), and loading a module may
+ *     allocate device memory and synchronize.  Callers whose later calls must
+ *     never do either make one warm-up call per device first (or run with
+ *     CUDA_MODULE_LOADING=EAGER, which loads the image when the context is
+ *     created).
  *   - Every call on a device shares the one array: two calls whose work may
  *     overlap on the GPU (different streams, no ordering) race on it.  Calls
  *     on one stream are ordered and safe.  Nothing in the array needs to
@@ -248,6 +270,62 @@ BITNET_API bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* prob
 BITNET_API bitnet_status bitnet_i2s_quant_gemv_noalloc(const uint8_t* packed, int64_t N, int64_t K,
                                                        const float* X, int64_t M, float* Y,
                                                        int32_t* acc_or_null, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Block-64 formats ["ik_llama.cpp 运行 BitNet b1.58 2B 模型实战", section 5.2:
+ * iq2_bn about 2 bits and iq1_bn 1.625 bits per weight, iq2_bn_r4 = iq2_bn
+ * packed in groups of 4 rows; section 5.3: K a multiple of the block of 64;
+ * section 6: one row quantized at a time, IQ1_BN decoded with multiplies,
+ * adds and shifts; section 5.1: the conversion from I2_S goes through f32,
+ * i.e. bitnet_i2s_dequant_f32 then one of the packs below].  The page leaves
+ * the bits inside a block open; this library's layouts:
+ *   IQ2_BN: a block of 64 weights is 16 bytes, weight j in byte j % 16,
+ *     bits [7-2g : 6-2g] with g = j / 16, code = w + 1.  Row n is K/64 blocks;
+ *     N*K/4 code bytes are followed by N little-endian fp32 row scales
+ *     d_n = max_k |W[n,k]|, with w = clip(round_half_away(W/d_n), -1, 1).
+ *   IQ2_BN_R4 (r4 != 0; N a multiple of 4): block b of row 4G + r at byte
+ *     ((G*(K/64) + b)*4 + r)*16; row scales as IQ2_BN.
+ *   IQ1_BN: a block of 64 weights is 13 bytes; byte i < 12 holds weights
+ *     5i .. 5i+4, byte 12 weights 60 .. 63, as ceil(256 v / 243) with
+ *     v = sum_j (w_j + 1) 3^(4-j); row scales after the N*(K/64)*13 code
+ *     bytes, which must be a multiple of 4.
+ * Conventions as for I2_S (device pointers, asynchronous on `stream`,
+ * host-side argument checks); all buffers 16-byte aligned; K <= 131072.
+ */
+
+/* Size in bytes of an IQ2_BN or IQ2_BN_R4 tensor (0 for a bad shape). */
+BITNET_API size_t bitnet_iq2bn_bytes(int64_t N, int64_t K);
+
+/* Size in bytes of an IQ1_BN tensor (0 for a bad shape). */
+BITNET_API size_t bitnet_iq1bn_bytes(int64_t N, int64_t K);
+
+/* Pack fp32 W[N,K] into IQ2_BN (r4 == 0) or IQ2_BN_R4 (r4 != 0), one scale
+ * per row.  out: bitnet_iq2bn_bytes(N,K) bytes, fully written. */
+BITNET_API bitnet_status bitnet_iq2bn_pack(const float* W, int64_t N, int64_t K, int r4,
+                                           uint8_t* out, void* stream);
+
+/* IQ2_BN / IQ2_BN_R4 -> fp32 W_out[N,K] = w * d_n, exact. */
+BITNET_API bitnet_status bitnet_iq2bn_dequant_f32(const uint8_t* packed, int64_t N, int64_t K,
+                                                  int r4, float* W_out, void* stream);
+
+/* Pack fp32 W[N,K] into IQ1_BN, one scale per row.  out:
+ * bitnet_iq1bn_bytes(N,K) bytes, fully written.  N*(K/64) % 4 == 0. */
+BITNET_API bitnet_status bitnet_iq1bn_pack(const float* W, int64_t N, int64_t K, uint8_t* out,
+                                           void* stream);
+
+/* IQ1_BN -> fp32 W_out[N,K] = w * d_n, exact. */
+BITNET_API bitnet_status bitnet_iq1bn_dequant_f32(const uint8_t* packed, int64_t N, int64_t K,
+                                                  float* W_out, void* stream);
+
+/* Decode matmul on IQ2_BN_R4 weights, M = 1 or 2 tokens, K <= 8192
+ * [P5 section 5 figure: add, subtract or skip per ternary weight; the row's
+ * scale in place of the tensor's]:
+ *   acc[m,n] = sum_k w[n,k] * Xq[m,k] (exact int32),
+ *   Y[m,n] = ((float)acc[m,n] * xs[m]) * d_n.
+ * Layouts of Xq, xs, Y and acc_or_null as bitnet_i2s_gemv. */
+BITNET_API bitnet_status bitnet_iq2bn_r4_gemv(const uint8_t* packed, int64_t N, int64_t K,
+                                              const int8_t* Xq, const float* xs, int64_t M,
+                                              float* Y, int32_t* acc_or_null, void* stream);
 
 /* Waits for all work on the current device, then returns
  * BITNET_ERR_DEVICE_TIMEOUT if any kernel of this library gave up on a

@@ -52,3 +52,31 @@ def column_sum_identity(acc, xq, t):
     want = (xq.to(torch.int64) * colsum[None, :]).sum(dim=1)  # [M]
     got = acc.to(torch.int64).sum(dim=1)
     return torch.equal(got.cpu(), want.cpu())
+
+
+# Guard bands: outputs the GPU tests hand to the library are views into a
+# larger buffer whose bytes before and after the view hold a known pattern,
+# so a write past a ragged edge into a neighbouring allocation fails a test
+# even though the in-range comparison cannot see it.
+GUARD_BYTES = 512
+GUARD_FILL = 0xA5
+
+
+def guarded_empty(shape, dtype, device="cuda"):
+    """(view, buffer): a contiguous `shape` view with GUARD_BYTES of pattern on
+    each side.  The view starts 512 bytes into the buffer, so it keeps the
+    buffer's 256-byte alignment."""
+    numel = 1
+    for s in shape:
+        numel *= int(s)
+    esize = torch.empty((), dtype=dtype).element_size()
+    g = GUARD_BYTES // esize
+    buf = torch.empty(numel + 2 * g, dtype=dtype, device=device)
+    buf.view(torch.uint8).fill_(GUARD_FILL)
+    return buf[g:g + numel].view(*shape), buf
+
+
+def guards_intact(buf) -> bool:
+    """True if both guard bands of a guarded_empty buffer still hold the pattern."""
+    b = buf.view(torch.uint8).cpu()
+    return bool((b[:GUARD_BYTES] == GUARD_FILL).all() and (b[-GUARD_BYTES:] == GUARD_FILL).all())

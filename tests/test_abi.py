@@ -132,13 +132,34 @@ def test_gemv_batched_workspace_checks_on_host(i2s):
     assert "workspace" in i2s.bitnet_last_error()
 
 
-def test_batched_workspace_includes_the_work_counters(i2s):
+def _align(v):
+    return (v + 255) // 256 * 256
+
+
+def test_batched_workspace_layout(i2s):
+    """Activation slots (M x K int8 and M scales, each 256-byte aligned), then
+    the decode tail: one work counter per decode launch and, for up to two
+    tokens, per launch 512 x 4 split arrival counters and 512 x 128 x M
+    split partial sums."""
     ks = [2560, 2560, 2560, 2560, 2560, 2560, 6912] * 30
     arr = (i2s.Problem * len(ks))()
     for i, k in enumerate(ks):
         arr[i] = i2s.Problem(A, 640, k, A, A, None)
-    slots = sum(i2s.bitnet_i2s_quant_gemv_workspace_bytes(1, k) for k in ks)
-    need = i2s.lib.bitnet_i2s_quant_gemv_batched_workspace_bytes(arr, len(ks), 1)
-    # one 256-byte block of counters (three decode launches at most) after the slots
-    assert need == slots + 256
+    launches = -(-len(ks) // 160) + 1  # one more: long-K and short-K problems launch apart
+    for m in (1, 2, 3, 16):
+        slots = sum(_align(m * k) + _align(4 * m) for k in ks)
+        tail = _align(4 * (launches + (launches * 512 * 4 if m <= 2 else 0)))
+        if m <= 2:
+            tail += _align(4 * launches * 512 * 128 * m)
+        need = i2s.lib.bitnet_i2s_quant_gemv_batched_workspace_bytes(arr, len(ks), m)
+        assert need == slots + tail, m
     assert i2s.lib.bitnet_i2s_quant_gemv_batched_workspace_bytes(arr, 0, 1) == 0
+    # the single fused call uses the batched layout for one problem
+    one = (i2s.Problem * 1)()
+    one[0] = i2s.Problem(A, 640, 2560, A, A, None)
+    for m in (1, 2, 5, 127):
+        assert (i2s.bitnet_i2s_quant_gemv_workspace_bytes(m, 2560) ==
+                i2s.lib.bitnet_i2s_quant_gemv_batched_workspace_bytes(one, 1, m))
+    # the pre-quantized batched call sizes its split area for two tokens
+    assert i2s.bitnet_i2s_gemv_batched_workspace_bytes(210) == (
+        _align(4 * (launches + launches * 512 * 4)) + _align(4 * launches * 512 * 128 * 2))
