@@ -1,21 +1,33 @@
 #!/usr/bin/env python
 """Benchmark of the I2_S ternary x int8 matmul on B200.
 
-Default workload (the JSON line's `value`): one decode step of the full
-BitNet-b1.58-2B-4T projection stack -- 30 layers x 7 projections (q/o
-2560x2560, k/v 640x2560, gate/up 6912x2560, down 2560x6912) = 210 fused
-activation-quant + ternary matmuls at batch 1, each with its own seeded
-fp32 input.  The 521 MB of packed weights stay resident in HBM; the working
-set is over 4x the 126 MB L2, so every step streams them from HBM.  One step
-is one replay of a CUDA graph holding one call of the public C ABI,
-bitnet_i2s_quant_gemv_batched, over the 210 problems (at batch 1 and 2 that
-is two launches: the activation quantizer and one persistent matmul).
-`value` is packed-weight GB/s over all ranks.
+Default workload (the JSON line's `value`, `--config 2`): one decode step of
+the full BitNet-b1.58-2B-4T projection stack -- 30 layers x 7 projections
+(q/o 2560x2560, k/v 640x2560, gate/up 6912x2560, down 2560x6912) = 210 fused
+activation-quant + ternary matmuls at batch 1, each with its own seeded fp32
+input.  The 521 MB of packed weights stay resident in HBM; the working set is
+over 4x the 126 MB L2, so every step streams them from HBM.  One step is one
+replay of a CUDA graph holding one call of the public C ABI,
+bitnet_i2s_quant_gemv_batched, over the 210 problems.  `value` is
+packed-weight GB/s over all ranks.
 
-Other measurements land in `extra`: the same stack as 210 separate
-bitnet_i2s_quant_gemv calls, the stack at batch 2, 4 and 16, the prefill
-GEMM (gate/up/down at M = 512 and 2048) in TOPS, and the single k_proj GEMV
-latency.
+`--config` picks another workload for the line (each streams more than L2
+per step, or rotates over distinct copies that together do):
+  0  one k_proj GEMV (640x2560, batch 1): 1231 distinct packed copies per
+     step in one batched fused call, plus the latency of a single call
+  1  one layer's 7 projections at batch 1 with 1 % x20 outlier channels,
+     rotated over 16 distinct copies of the layer, one call per step
+  2  the 30-layer stack (default), at --batch tokens
+  3  prefill GEMM: gate/up 6912x2560 and down 2560x6912 at --batch tokens
+     (default 2048) in one fused call per step; value in TOPS
+  4  a large BitNet-style layer (hidden 8192, ffn 28672), two copies at
+     batch 1 (GB/s), or one copy at --batch 64 (GB/s and TOPS)
+
+Secondary measurements (default run only) land in `extra`: the stack as 210
+separate calls; as a dependency-staged decode step (120 ordered calls, each
+stage reading the previous stage's output); a sustained run of the headline
+step over about a second with its clocks; the stack at batch 2, 4 and 16;
+prefill TOPS; the other configs' figures.
 
 Multi-GPU (`--gpus N` under torchrun): every rank holds a replica of the
 weights and runs its own token batch (data parallel, weak scaling); there is
@@ -45,12 +57,14 @@ FALLBACK_BF16_TFLOPS = 1590.0
 NOMINAL_INT8_OVER_BF16 = 2.0  # 4.5 POPS int8 dense / 2.25 PFLOP/s bf16 dense
 DECODE_BATCH = 160  # problems per launch of the decode kernel
 MMA_BATCH = 96  # problems per launch of the tensor-core kernel
+L2_BYTES = 126e6
 # (N, K) of the seven projections of one BitNet-b1.58-2B-4T block
 STACK_SHAPES = [(2560, 2560), (640, 2560), (640, 2560), (2560, 2560), (6912, 2560), (6912, 2560),
                 (2560, 6912)]
 TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "i2s_gemv_dp4a_stack_batch1.md")
 DECODE_SOURCES = [os.path.join(ROOT, "i2_mpgemm_b200", "csrc", f)
                   for f in ("gemv_kernel.cuh", "ptx.cuh")]
+DEFAULT_BATCH = {0: 1, 1: 1, 2: 1, 3: 2048, 4: 1}
 
 
 # ------------------------------------------------------------------ setup
@@ -61,7 +75,10 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--batch", type=int, default=1, help="decode tokens per step (1..64)")
+    ap.add_argument("--config", type=int, choices=[0, 1, 2, 3, 4], default=2,
+                    help="workload (see the module docstring); 2 is the 30-layer stack")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="tokens per step (default: 1, or 2048 for --config 3)")
     ap.add_argument("--layers", type=int, default=30)
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -69,7 +86,10 @@ def parse_args(argv=None):
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the gate 6912x2560 prefill GEMM at M=2048 (a small case "
                          "for profiling the tensor-core kernel) and print its own line")
-    return ap.parse_args(argv)
+    args = ap.parse_args(argv)
+    if args.batch is None:
+        args.batch = DEFAULT_BATCH[args.config]
+    return args
 
 
 def dist_env():
@@ -174,6 +194,7 @@ class ClockSampler:
     def __init__(self, gpu_id: str | None):
         self.proc = None
         self.gpu_id = gpu_id
+        self.lines = []
 
     def __enter__(self):
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -201,25 +222,35 @@ class ClockSampler:
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
         return False
 
-    def summary(self):
-        sm, mx, reasons = [], [], set()
+    def samples(self):
+        """[(sm_mhz, max_mhz, power_w, {reasons active})] per sample."""
+        out = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for name, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
+            try:
+                pw = float(parts[3])
+            except ValueError:
+                pw = float("nan")
+            reasons = {n for n, v in zip(names, parts[5:9]) if v.lower().startswith("active")}
+            out.append((sm, mx, pw, reasons))
+        return out
+
+    def summary(self):
+        s = self.samples()
+        if not s:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        reasons = set()
+        for *_, r in s:
+            reasons |= r
+        return {"sm_mhz": statistics.median(x[0] for x in s), "sm_max_mhz": max(x[1] for x in s),
+                "samples": len(s), "reasons": sorted(reasons)}
 
 
 def gpu_uuid(torch, device_index: int) -> str | None:
@@ -235,42 +266,57 @@ def gpu_uuid(torch, device_index: int) -> str | None:
 class Problem:
     """One projection: resident packed weights plus views of the step buffers."""
 
-    def __init__(self, i2s, torch, n, k, m, w, x, y):
+    def __init__(self, i2s, torch, n, k, m, w, x, y, packed=None):
         self.n, self.k, self.m = n, k, m
-        self.packed = i2s.bitnet_i2s_pack(w.cuda())
+        self.packed = i2s.bitnet_i2s_pack(w.cuda()) if packed is None else packed
         self.packed_bytes = n * k // 4
         self.x, self.y = x, y
         self.ws = torch.empty(i2s.bitnet_i2s_quant_gemv_workspace_bytes(m, k), dtype=torch.uint8,
                               device="cuda")
 
 
-class Stack:
-    """The projection stack with every input in one device buffer and every
-    output in another (each problem's X and Y are views), so an end-to-end
-    step moves its inputs and outputs with one copy each way."""
+class Buffers:
+    """Every step input in one device buffer and every output in another
+    (each problem's X and Y are views), with pinned host copies, so an
+    end-to-end step moves a step's inputs and outputs with one copy each."""
 
-    def __init__(self, i2s, torch, inputs, layers: int, m: int, act_seed_offset: int):
-        shapes = [(layer, idx, p) for layer in range(layers)
-                  for idx, p in enumerate(inputs.projections_2b())]
-        x_total = sum(m * p.k for _, _, p in shapes)
-        y_total = sum(m * p.n for _, _, p in shapes)
+    def __init__(self, torch, x_total: int, y_total: int):
         self.x_dev = torch.empty(x_total, dtype=torch.float32, device="cuda")
         self.y_dev = torch.empty(y_total, dtype=torch.float32, device="cuda")
         self.x_host = torch.empty(x_total, dtype=torch.float32).pin_memory()
         self.y_host = torch.empty(y_total, dtype=torch.float32).pin_memory()
+        self.xo = self.yo = 0
+
+    def take(self, m, k, n):
+        x = self.x_dev[self.xo:self.xo + m * k].view(m, k)
+        y = self.y_dev[self.yo:self.yo + m * n].view(m, n)
+        xh = self.x_host[self.xo:self.xo + m * k]
+        self.xo += m * k
+        self.yo += m * n
+        return x, y, xh
+
+
+class Stack:
+    """The projection stack (layers x 7 problems) in one Buffers."""
+
+    def __init__(self, i2s, torch, inputs, layers: int, m: int, act_seed_offset: int,
+                 outliers: bool = False, seed_fn=None):
+        seed_fn = seed_fn or inputs.seed_stack
+        shapes = [(layer, idx, p) for layer in range(layers)
+                  for idx, p in enumerate(inputs.projections_2b())]
+        self.buf = Buffers(torch, sum(m * p.k for _, _, p in shapes),
+                           sum(m * p.n for _, _, p in shapes))
         self.probs = []
-        xo = yo = 0
         for layer, idx, p in shapes:
-            seed = inputs.seed_stack(layer, idx)
+            seed = seed_fn(layer, idx)
             w, _, _ = inputs.ternary_weights(p.n, p.k, seed)
-            xv = inputs.activations(m, p.k, seed + act_seed_offset)
-            self.x_host[xo:xo + m * p.k].copy_(xv.reshape(-1))
-            x = self.x_dev[xo:xo + m * p.k].view(m, p.k)
-            y = self.y_dev[yo:yo + m * p.n].view(m, p.n)
+            x, y, xh = self.buf.take(m, p.k, p.n)
+            xh.copy_(inputs.activations(m, p.k, seed + act_seed_offset, outliers=outliers)
+                     .reshape(-1))
             self.probs.append(Problem(i2s, torch, p.n, p.k, m, w, x, y))
-            xo += m * p.k
-            yo += m * p.n
             del w
+        self.x_dev, self.y_dev = self.buf.x_dev, self.buf.y_dev
+        self.x_host, self.y_host = self.buf.x_host, self.buf.y_host
         self.x_dev.copy_(self.x_host)
         torch.cuda.synchronize()
 
@@ -312,27 +358,31 @@ def capture(torch, fn):
 
 def time_replays(torch, g, steps: int, warmup: int, before=None, after=None,
                  collective: bool = True) -> float:
-    """Milliseconds per replay, CUDA events on the replay stream.  With
-    `collective`, every rank must call it (barriers before and after);
-    rank-0-only measurements pass collective=False."""
-    for _ in range(warmup):
+    """Milliseconds per step, CUDA events on the replay stream.  `g` is one
+    graph (replayed every step) or a list of graphs (step i replays
+    g[i % len(g)]; `before`/`after` then get i).  With `collective`, every
+    rank must call it (barriers before and after); rank-0-only measurements
+    pass collective=False."""
+    graphs = g if isinstance(g, list) else [g]
+    rot = isinstance(g, list)
+
+    def one(i):
         if before:
-            before()
-        g.replay()
+            before(i) if rot else before()
+        graphs[i % len(graphs)].replay()
         if after:
-            after()
+            after(i) if rot else after()
+
+    for i in range(warmup):
+        one(i)
     torch.cuda.synchronize()
     if collective:
         barrier()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
-    for _ in range(steps):
-        if before:
-            before()
-        g.replay()
-        if after:
-            after()
+    for i in range(steps):
+        one(i)
     end.record()
     end.synchronize()
     torch.cuda.synchronize()
@@ -341,69 +391,135 @@ def time_replays(torch, g, steps: int, warmup: int, before=None, after=None,
     return start.elapsed_time(end) / steps
 
 
-def matmul_kernel_time(i2s, torch, probs, reps: int = 20):
+def matmul_kernel_time(i2s, torch, plans_probs, reps: int = 20):
     """Average device time of the matmul launch(es) of one step, CUDA events
     on the launching stream, with the activations quantized beforehand so the
-    timed region holds only the matmul kernel.  Returns (ms per step,
-    launches per step, algorithmic bytes per step)."""
-    qs = [i2s.bitnet_act_quant_i8(p.x) for p in probs]
+    timed region holds only the matmul kernels (and, for the decode kernel,
+    the one-warp reset of its work counters).  `plans_probs` is a list of
+    steps, each a list of Problem; the timed loop rotates over them.
+    Returns (ms per step, launches per step, algorithmic bytes per step)."""
+    plans, nbytes = [], 0
+    for probs in plans_probs:
+        qs = [i2s.bitnet_act_quant_i8(p.x) for p in probs]
+        m = probs[0].m
+        plans.append(i2s.BatchedGemv([(p.packed, p.n, p.k, q, s, p.y, None)
+                                      for p, (q, s) in zip(probs, qs)], m))
+        nbytes += sum(p.packed_bytes + 4 + p.m * p.k + 4 * p.m + 4 * p.m * p.n for p in probs)
+    probs = plans_probs[0]
     m = probs[0].m
-    plan = i2s.BatchedGemv([(p.packed, p.n, p.k, q, s, p.y, None)
-                            for p, (q, s) in zip(probs, qs)], m)
-    # The decode kernel takes up to DECODE_BATCH problems per launch (M <= 2,
-    # K <= 8192, or M = 1 with K <= 30720), the tensor-core kernel up to
-    # MMA_BATCH; the call also zeroes
-    # the decode launches' work counters (one memset, inside the timed region).
     small = [p for p in probs if (m <= 2 and p.k <= 8192) or (m == 1 and p.k <= 30720)]
     launches = -(-len(small) // DECODE_BATCH) + -(-(len(probs) - len(small)) // MMA_BATCH)
     for _ in range(3):
-        plan.run()
+        for pl in plans:
+            pl.run()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(reps):
-        plan.run()
+    for i in range(reps * len(plans)):
+        plans[i % len(plans)].run()
     b.record(stream)
     b.synchronize()
-    ms = a.elapsed_time(b) / reps
-    nbytes = sum(p.packed_bytes + 4 + p.m * p.k + 4 * p.m + 4 * p.m * p.n for p in probs)
-    return ms, launches, nbytes
+    ms = a.elapsed_time(b) / (reps * len(plans))
+    return ms, launches, nbytes / len(plans)
 
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_layer_sample(inputs, m: int):
+def oracle_layer_sample(inputs, m: int, outliers: bool = False, seed_fn=None):
     """One layer's seven projections packed by the oracle, with inputs."""
     import oracle
+    seed_fn = seed_fn or inputs.seed_stack
     sample = []
     for idx, p in enumerate(inputs.projections_2b()):
-        seed = inputs.seed_stack(0, idx)
+        seed = seed_fn(0, idx)
         w, _, _ = inputs.ternary_weights(p.n, p.k, seed)
-        x = inputs.activations(m, p.k, seed)
+        x = inputs.activations(m, p.k, seed, outliers=outliers)
         sample.append((oracle.pack(w.numpy()), p.n, p.k, x.numpy()))
     return sample
 
 
-def oracle_layer_seconds(sample) -> float:
+def oracle_sample(inputs, config: int, m: int):
+    """The bounded sample of a config's workload that the oracle runs: a list
+    of (packed, n, k, x) problems, the unit of the rate, the work per pass
+    in that unit's base (bytes or int ops), and a description."""
+    import oracle
+    if config == 0:
+        w, _, _ = inputs.ternary_weights(640, 2560, inputs.seed_single())
+        x = inputs.activations(m, 2560, inputs.seed_single())
+        s = [(oracle.pack(w.numpy()), 640, 2560, x.numpy())]
+        return s, "GB/s", 640 * 2560 // 4, f"the k_proj 640x2560 GEMV at batch {m}"
+    if config in (1, 2):
+        outl = config == 1
+        seed_fn = (lambda layer, idx: inputs.seed_layer(idx)) if outl else None
+        s = oracle_layer_sample(inputs, m, outliers=outl, seed_fn=seed_fn)
+        what = ("the layer's 7 projections with outliers" if outl else
+                "one layer's 7 projections (1/30 of the stack)")
+        return s, "GB/s", sum(n * k // 4 for _, n, k, _ in s), f"{what} at batch {m}"
+    if config == 3:
+        tok = min(m, 4)  # a few of the prompt's tokens through gate, up and down
+        s = []
+        for idx, (n, k) in enumerate([(6912, 2560), (6912, 2560), (2560, 6912)]):
+            seed = inputs.seed_prefill(idx)
+            w, _, _ = inputs.ternary_weights(n, k, seed)
+            x = inputs.activations(m, k, seed)[:tok]
+            s.append((oracle.pack(w.numpy()), n, k, x.numpy()))
+        return s, "TOPS", sum(2 * tok * n * k for _, n, k, _ in s), \
+            f"the first {tok} of the {m} tokens through gate, up and down"
+    p = inputs.projections_large()[6]  # down 8192 x 28672
+    w, _, _ = inputs.ternary_weights(p.n, p.k, inputs.seed_large(6))
+    x = inputs.activations(1, p.k, inputs.seed_large(6))
+    return [(oracle.pack(w.numpy()), p.n, p.k, x.numpy())], "GB/s", p.n * p.k // 4, \
+        "the large layer's down projection 8192x28672 at batch 1"
+
+
+def oracle_pass(sample):
+    """One pass of the oracle over a sample: (seconds, outputs)."""
     import oracle
     t0 = time.perf_counter()
-    for packed, n, k, x in sample:
-        oracle.quant_gemm(packed, n, k, x)
-    return time.perf_counter() - t0
+    ys = [oracle.quant_gemm(packed, n, k, x)[0] for packed, n, k, x in sample]
+    return time.perf_counter() - t0, ys
 
 
-def cpu_baseline(inputs, m: int, budget_s: float):
-    sample = oracle_layer_sample(inputs, m)
-    layer_bytes = sum(n * k // 4 for _, n, k, _ in sample)
-    done, spent = 0, 0.0
-    while spent < budget_s:
-        spent += oracle_layer_seconds(sample)
+def rate(work: float, seconds: float, unit: str) -> float:
+    return work / seconds / (1e9 if unit == "GB/s" else 1e12)
+
+
+def cpu_baseline(inputs, config: int, m: int, budget_s: float, gpu_outputs=None):
+    """The oracle, one thread, on the config's bounded sample for about
+    `budget_s`.  With `gpu_outputs` (the timed step's outputs of the same
+    sample problems, host arrays), the first pass's outputs are compared
+    with them at the tests' tolerance, and the verdict is reported."""
+    sample, unit, work, what = oracle_sample(inputs, config, m)
+    done, spent, ys = 0, 0.0, None
+    while spent < budget_s or done == 0:
+        dt, out = oracle_pass(sample)
+        ys = ys or out
+        spent += dt
         done += 1
-    return {"value": round(done * layer_bytes / spent / 1e9, 6), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{done} passes over one layer's 7 projections at batch {m} "
-                      f"(scalar C oracle, one thread, {spent:.1f} s)"}
+    res = {"value": round(rate(done * work, spent, unit), 6), "unit": unit, "cores": 1,
+           "kind": "oracle",
+           "sample": f"{done} passes over {what} (scalar C oracle, one thread, {spent:.1f} s)"}
+    if gpu_outputs is not None:
+        res["parity"] = compare_outputs(gpu_outputs, ys)
+    return res
+
+
+def compare_outputs(got, want):
+    """Element-wise comparison of the GPU step's outputs with the oracle's:
+    within 1e-5 relative error and exactly zero where the oracle's is."""
+    import numpy as np
+    worst, count, ok = 0.0, 0, True
+    for g, w in zip(got, want):
+        g = np.asarray(g, dtype=np.float64).reshape(w.shape)
+        w = np.asarray(w, dtype=np.float64)
+        zero = w == 0
+        ok = ok and bool(np.all(g[zero] == 0))
+        if (~zero).any():
+            worst = max(worst, float(np.max(np.abs(g[~zero] - w[~zero]) / np.abs(w[~zero]))))
+        count += w.size
+    ok = ok and worst <= 1e-5
+    return {"parity_ok": ok, "outputs_compared": count, "max_rel_err": worst}
 
 
 _WORKER_SAMPLE = None
@@ -448,23 +564,21 @@ def run_reference(args):
         return 0
     from i2_mpgemm_b200 import inputs
     m = args.batch
-    sample = oracle_layer_sample(inputs, m)
-    layer_bytes = sum(n * k // 4 for _, n, k, _ in sample)
+    sample, unit, work, what = oracle_sample(inputs, args.config, m)
     for _ in range(args.warmup):
-        oracle_layer_seconds(sample)
-    secs = [oracle_layer_seconds(sample) for _ in range(args.steps)]
+        oracle_pass(sample)
+    secs = [oracle_pass(sample)[0] for _ in range(args.steps)]
     total = sum(secs)
-    value = args.steps * layer_bytes / total / 1e9
+    value = rate(args.steps * work, total, unit)
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1000 * total / args.steps, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": workload_config(args.layers, m),
-        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: one layer's 7 projections at batch {m} "
-                                   "(1/30 of the stack), scalar C oracle, one thread"},
-        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": DATA,
+        "config": workload_config(args.config, m, args.layers, args.gpus),
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {what}, scalar C oracle, one thread"},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -472,17 +586,64 @@ def run_reference(args):
     return 0
 
 
-def workload_config(layers: int, m: int):
+DATA = ("synthetic (seeded ternary weights p=.25/.5/.25 x U(0.5,2) scale, N(0,1) activations)")
+
+
+def workload_config(config: int, m: int, layers: int = 30, world: int = 1):
+    """The `config` object of the JSON line, identical for both arms."""
+    par = f"replicas x{world} (data parallel, no collective)"
+    if config == 0:
+        copies = kproj_copies()
+        return {"workload": (f"k_proj GEMV 640x2560 at batch {m}, fused act-quant + I2_S matmul: "
+                             f"{copies} distinct packed copies per step in one batched call"),
+                "global_batch": m * world, "packed_bytes_per_step": copies * 640 * 2560 // 4,
+                "l2": "inputs larger than L2: the copies total over 4x L2",
+                "parallelism": par}
+    if config == 1:
+        return {"workload": ("one BitNet-b1.58-2B-4T layer's 7 projections at batch "
+                             f"{m}, 1% outlier channels x20, fused act-quant + I2_S matmul, "
+                             f"one call per step rotating over {LAYER_COPIES} layer copies"),
+                "global_batch": m * world,
+                "packed_bytes_per_step": sum(n * k // 4 for n, k in STACK_SHAPES),
+                "l2": f"rotation over {LAYER_COPIES} distinct copies ({LAYER_COPIES} x 17.4 MB) "
+                      "exceeds L2",
+                "parallelism": par}
+    if config == 3:
+        return {"workload": (f"prefill GEMM at M={m}: gate/up 6912x2560 and down 2560x6912, "
+                             "fused act-quant + tcgen05 int8 matmul, one batched call per step"),
+                "global_batch": m * world,
+                "int_ops_per_step": 2 * m * (2 * 6912 * 2560 + 2560 * 6912),
+                "l2": "weights and activations L2-resident: tensor-bound by design",
+                "parallelism": par}
+    if config == 4:
+        copies = 2 if m == 1 else 1
+        return {"workload": (f"large BitNet-style layer (hidden 8192, ffn 28672), {copies} "
+                             f"copies of its 7 projections at batch {m}, fused act-quant + I2_S "
+                             "matmul in one batched call per step"),
+                "global_batch": m * world,
+                "packed_bytes_per_step": copies * LARGE_LAYER_BYTES,
+                "l2": "inputs larger than L2 (214 MB per copy)",
+                "parallelism": par}
     return {
         "workload": (f"BitNet-b1.58-2B-4T projection stack, {layers} layers x 7 "
                      "(q/o 2560x2560, k/v 640x2560, gate/up 6912x2560, down 2560x6912), "
                      f"decode batch {m}, fused act-quant + I2_S matmul per projection"),
-        "global_batch": m,
+        "global_batch": m * world,
         "packed_bytes_per_step": layers * sum(n * k // 4 for n, k in STACK_SHAPES),
         "l2": "inputs larger than L2: each step streams all packed weights (521 MB for 30 "
               "layers) from HBM",
-        "parallelism": "replicas (data parallel, no collective)",
+        "parallelism": par,
     }
+
+
+LAYER_COPIES = 16
+# K of the problems of each of the four dependent calls of one layer
+STAGE_KS = [[2560] * 3, [2560], [2560] * 2, [6912]]
+LARGE_LAYER_BYTES = (2 * 8192 * 8192 + 2 * 1024 * 8192 + 3 * 28672 * 8192) // 4
+
+
+def kproj_copies() -> int:
+    return int(4 * L2_BYTES / (640 * 2560 // 4)) + 1
 
 
 # ----------------------------------------------------------------- extras
@@ -517,25 +678,225 @@ def int8_gemm_tops(torch):
         return None
 
 
-def gpu_ternary(torch, n: int, k: int, seed: int):
+def int8_peak(torch, peaks):
+    """(TOPS, source): the measured int8 GEMM, else bf16 burst x 2."""
+    measured = int8_gemm_tops(torch)
+    if measured:
+        return measured, "measured: torch._int_mm 8192^3 best of 10"
+    return (NOMINAL_INT8_OVER_BF16 * peaks["bf16_tflops"],
+            f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 ratio)")
+
+
+def gpu_ternary(torch, n: int, k: int, seed: int, scale=None):
     """Seeded ternary weights drawn on the device (same distribution as the
-    host generator: -1/0/+1 with p = .25/.5/.25 times s ~ U(0.5, 2)), for the
-    timing-only large layer whose host generation would take minutes."""
+    host generator: -1/0/+1 with p = .25/.5/.25, times s ~ U(0.5, 2) or the
+    given scale), for timing-only workloads whose host generation would take
+    minutes."""
     g = torch.Generator(device="cuda")
     g.manual_seed(seed)
     r = torch.randint(0, 4, (n, k), generator=g, device="cuda", dtype=torch.int32)
-    s = 0.5 + 1.5 * torch.rand((), generator=g, device="cuda")
+    s = 0.5 + 1.5 * torch.rand((), generator=g, device="cuda") if scale is None else scale
     return ((r == 3).float() - (r == 0).float()) * s
 
 
-def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
+class Workload:
+    """A config's timed work: `steps` is a list of steps, each a list of
+    Problem run by one batched fused call; step i of a run uses
+    steps[i % len(steps)].  All inputs sit in one Buffers."""
+
+    def __init__(self, i2s, torch, steps, buf, unit, work_per_step, launches_per_step):
+        self.i2s, self.torch = i2s, torch
+        self.steps, self.buf, self.unit = steps, buf, unit
+        self.work = work_per_step
+        self.launches = launches_per_step
+        self.plans = [stack_batch(i2s, probs) for probs in steps]
+        self.ranges = []  # per step: (x lo, x hi, y lo, y hi) in the buffers
+        for probs in steps:
+            xs = [p.x.data_ptr() for p in probs]
+            ys = [p.y.data_ptr() for p in probs]
+            xb, yb = buf.x_dev.data_ptr(), buf.y_dev.data_ptr()
+            xlo = (min(xs) - xb) // 4
+            xhi = max((p.x.data_ptr() - xb) // 4 + p.x.numel() for p in probs)
+            ylo = (min(ys) - yb) // 4
+            yhi = max((p.y.data_ptr() - yb) // 4 + p.y.numel() for p in probs)
+            self.ranges.append((xlo, xhi, ylo, yhi))
+
+    def graphs(self):
+        return [capture(self.torch, pl.run) for pl in self.plans]
+
+    def h2d(self, i):
+        lo, hi, _, _ = self.ranges[i % len(self.ranges)]
+        self.buf.x_dev[lo:hi].copy_(self.buf.x_host[lo:hi], non_blocking=True)
+
+    def d2h(self, i):
+        _, _, lo, hi = self.ranges[i % len(self.ranges)]
+        self.buf.y_host[lo:hi].copy_(self.buf.y_dev[lo:hi], non_blocking=True)
+
+    def io_bytes(self):
+        lo, hi, ylo, yhi = self.ranges[0]
+        return 4 * (hi - lo), 4 * (yhi - ylo)
+
+
+def problems_from_weights(i2s, torch, buf, specs, m):
+    """Problems of (packed or fp32 weights, n, k, x host) specs in `buf`."""
+    probs = []
+    for w_or_packed, n, k, xh in specs:
+        x, y, xhv = buf.take(m, k, n)
+        xhv.copy_(xh.reshape(-1))
+        if w_or_packed.dtype == torch.uint8:
+            probs.append(Problem(i2s, torch, n, k, m, None, x, y, packed=w_or_packed))
+        else:
+            probs.append(Problem(i2s, torch, n, k, m, w_or_packed, x, y))
+    return probs
+
+
+def build_workload(i2s, torch, inputs, config: int, m: int, layers: int, rank: int):
+    """The timed Workload of a config (each rank draws its own activations)."""
+    off = 7919 * rank
+    if config == 2:
+        st = Stack(i2s, torch, inputs, layers, m, act_seed_offset=off)
+        return Workload(i2s, torch, [st.probs], st.buf, "GB/s",
+                        sum(p.packed_bytes for p in st.probs),
+                        step_launches(m, [p.k for p in st.probs]))
+    if config == 1:
+        # LAYER_COPIES distinct copies of the layer (the same weights and
+        # inputs), one call per step over one copy
+        base = [(inputs.ternary_weights(p.n, p.k, inputs.seed_layer(idx))[0], p)
+                for idx, p in enumerate(inputs.projections_2b())]
+        xs = [inputs.activations(m, p.k, inputs.seed_layer(idx) + off, outliers=True)
+              for idx, p in enumerate(inputs.projections_2b())]
+        buf = Buffers(torch, LAYER_COPIES * sum(m * p.k for _, p in base),
+                      LAYER_COPIES * sum(m * p.n for _, p in base))
+        packs = [i2s.bitnet_i2s_pack(w.cuda()) for w, _ in base]
+        steps = []
+        for c in range(LAYER_COPIES):
+            specs = [(pk if c == 0 else pk.clone(), p.n, p.k, x)
+                     for pk, (_, p), x in zip(packs, base, xs)]
+            steps.append(problems_from_weights(i2s, torch, buf, specs, m))
+        buf.x_dev.copy_(buf.x_host)
+        return Workload(i2s, torch, steps, buf, "GB/s", sum(n * k // 4 for n, k in STACK_SHAPES),
+                        step_launches(m, [p.k for _, p in base]))
+    if config == 0:
+        copies = kproj_copies()
+        w, _, _ = inputs.ternary_weights(640, 2560, inputs.seed_single())
+        x = inputs.activations(m, 2560, inputs.seed_single() + off)
+        pk = i2s.bitnet_i2s_pack(w.cuda())
+        buf = Buffers(torch, copies * m * 2560, copies * m * 640)
+        specs = [(pk if c == 0 else pk.clone(), 640, 2560, x) for c in range(copies)]
+        probs = problems_from_weights(i2s, torch, buf, specs, m)
+        buf.x_dev.copy_(buf.x_host)
+        return Workload(i2s, torch, [probs], buf, "GB/s", copies * 640 * 2560 // 4,
+                        step_launches(m, [2560] * copies))
+    if config == 3:
+        shapes = [(6912, 2560), (6912, 2560), (2560, 6912)]
+        buf = Buffers(torch, sum(m * k for _, k in shapes), sum(m * n for n, _ in shapes))
+        specs = []
+        for idx, (n, k) in enumerate(shapes):
+            seed = inputs.seed_prefill(idx)
+            specs.append((inputs.ternary_weights(n, k, seed)[0], n, k,
+                          inputs.activations(m, k, seed + off)))
+        probs = problems_from_weights(i2s, torch, buf, specs, m)
+        buf.x_dev.copy_(buf.x_host)
+        return Workload(i2s, torch, [probs], buf, "TOPS",
+                        sum(2.0 * m * n * k for n, k in shapes), step_launches(m, [2560, 2560, 6912]))
+    # config 4: device-drawn weights (host generation of 1.7 G weights would take minutes)
+    large = inputs.projections_large()
+    copies = 2 if m == 1 else 1
+    buf = Buffers(torch, copies * sum(m * p.k for p in large), copies * sum(m * p.n for p in large))
+    packs = []
+    for idx, p in enumerate(large):
+        w = gpu_ternary(torch, p.n, p.k, inputs.seed_large(idx))
+        packs.append(i2s.bitnet_i2s_pack(w))
+        del w
+    torch.cuda.empty_cache()
+    specs = []
+    for c in range(copies):
+        for idx, p in enumerate(large):
+            specs.append((packs[idx] if c == 0 else packs[idx].clone(), p.n, p.k,
+                          inputs.activations(m, p.k, inputs.seed_large(idx) + off)))
+    probs = problems_from_weights(i2s, torch, buf, specs, m)
+    buf.x_dev.copy_(buf.x_host)
+    return Workload(i2s, torch, [probs], buf, "GB/s", copies * LARGE_LAYER_BYTES,
+                    step_launches(m, [p.k for p in large] * copies))
+
+
+def staged_stack(i2s, torch, inputs, layers: int, m: int):
+    """A dependency-staged decode step over the stack's shapes: per layer
+    four ordered calls -- q+k+v on the layer input, o on q's output, gate+up
+    on o's output, down on gate's output, whose output is the next layer's
+    input -- 4 x layers batched fused calls, each stage reading what the one
+    before it wrote.  Weights are drawn on the device with a per-tensor scale
+    of 1/sqrt(K/2), so that the values passed from stage to stage keep their
+    size over 120 stages instead of overflowing; the matmul is the same.
+    Returns (list of BatchedQuantGemv in order, packed bytes per step)."""
+    P = {p.name: p for p in inputs.projections_2b()}
+    keep, calls, nbytes = [], [], 0
+    h = torch.randn((m, P["q"].k), generator=torch.Generator(device="cuda").manual_seed(5),
+                    device="cuda")
+    keep.append(h)
+    for layer in range(layers):
+        def proj(name, idx):
+            p = P[name]
+            w = gpu_ternary(torch, p.n, p.k, inputs.seed_stack(layer, idx),
+                            scale=float((p.k / 2) ** -0.5))
+            pk = i2s.bitnet_i2s_pack(w)
+            keep.append(pk)
+            return pk, p
+        def out(p):
+            y = torch.empty((m, p.n), device="cuda")
+            keep.append(y)
+            return y
+        (q, pq), (k_, pk_), (v, pv) = proj("q", 0), proj("k", 1), proj("v", 2)
+        yq, yk, yv = out(pq), out(pk_), out(pv)
+        calls.append(i2s.BatchedQuantGemv([(q, pq.n, pq.k, h, yq, None),
+                                           (k_, pk_.n, pk_.k, h, yk, None),
+                                           (v, pv.n, pv.k, h, yv, None)], m))
+        o, po = proj("o", 3)
+        yo = out(po)
+        calls.append(i2s.BatchedQuantGemv([(o, po.n, po.k, yq, yo, None)], m))
+        (g, pg), (u, pu) = proj("gate", 4), proj("up", 5)
+        yg, yu = out(pg), out(pu)
+        calls.append(i2s.BatchedQuantGemv([(g, pg.n, pg.k, yo, yg, None),
+                                           (u, pu.n, pu.k, yo, yu, None)], m))
+        d, pd = proj("down", 6)
+        h = out(pd)
+        calls.append(i2s.BatchedQuantGemv([(d, pd.n, pd.k, yg, h, None)], m))
+        nbytes += sum(n * k // 4 for n, k in STACK_SHAPES)
+    torch.cuda.empty_cache()
+    return calls, nbytes, keep
+
+
+def extra_measurements(i2s, torch, inputs, args, work, g_head, peaks):
     out = {}
-    # int8 dense tensor peak: the library int8 GEMM measured here, else the
-    # measured bf16 burst peak times the nominal int8/bf16 ratio of 2
-    derived = 2.0 * peaks["bf16_tflops"]
-    measured = int8_gemm_tops(torch)
-    int8_tops = measured if measured else derived
-    # the batch-1 stack as 210 separate fused calls (420 launches per step)
+    steps = args.steps
+    int8_tops, int8_src = int8_peak(torch, peaks)
+    out["int8_peak_TOPS"] = round(int8_tops, 1)
+    out["int8_peak_source"] = int8_src
+    # sustained: the headline step replayed for about a second, clocks sampled
+    ms_one = time_replays(torch, g_head, 20, 3, collective=False)
+    n_sus = max(200, int(1000.0 / max(ms_one, 1e-3)))
+    with ClockSampler(gpu_uuid(torch, torch.cuda.current_device())) as clk:
+        ms = time_replays(torch, g_head, n_sus, 3, collective=False)
+    samp = clk.samples()
+    sus = {"steps": n_sus, "seconds": round(n_sus * ms / 1000, 3), "ms_per_step": round(ms, 4),
+           "packed_GBps": round(work.work / ms / 1e6, 1),
+           "frac_of_hbm_measured": round(work.work / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    if samp:
+        mhz = [s[0] for s in samp]
+        med = statistics.median(mhz)
+        bins = {}
+        for s in mhz:
+            key = f"{int(s // 100) * 100}-{int(s // 100) * 100 + 99}"
+            bins[key] = bins.get(key, 0) + 1
+        sus.update({"clock_samples": len(samp), "sm_mhz_median": med,
+                    "sm_mhz_bins": dict(sorted(bins.items())),
+                    "power_w_median": statistics.median(s[2] for s in samp),
+                    "reasons": sorted(set().union(*[s[3] for s in samp])),
+                    "ms_x_median_mhz": round(ms * med, 2)})
+    out["sustained"] = sus
+    probs1 = work.steps[0]
+    m1 = probs1[0].m
+    # the stack as 210 separate fused calls (420 launches per step)
     g = capture(torch, lambda: stack_step(i2s, probs1))
     ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
     nbytes = sum(p.packed_bytes for p in probs1)
@@ -543,15 +904,29 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
                                     "packed_GBps": round(nbytes / ms / 1e6, 1),
                                     "launches_per_step": 2 * len(probs1)}
     del g
+    # dependency-staged decode: 120 ordered calls per step
+    for m in (1, 16):
+        calls, sbytes, keep = staged_stack(i2s, torch, inputs, args.layers, m)
+        g = capture(torch, lambda: [c.run() for c in calls])
+        ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
+        out[f"stack_staged_batch{m}"] = {
+            "calls_per_step": len(calls), "ms_per_step": round(ms, 4),
+            "packed_GBps": round(sbytes / ms / 1e6, 1),
+            "frac_of_hbm_measured": round(sbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
+            "tokens_per_s": round(m * 1000.0 / ms, 1),
+            "launches_per_step": args.layers * sum(step_launches(m, ks) for ks in STAGE_KS)}
+        del g, calls, keep
+        torch.cuda.empty_cache()
     # the stack at batch 2, 4 and 16 (one batched call per step)
     for m in (2, 4, 16):
-        probs = build_stack(i2s, torch, inputs, 30, m, 0)
+        probs = build_stack(i2s, torch, inputs, args.layers, m, 0)
         plan = stack_batch(i2s, probs)
         g = capture(torch, plan.run)
         ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
         nbytes = sum(p.packed_bytes for p in probs)
         out[f"stack_batch{m}"] = {"ms_per_step": round(ms, 4), "packed_GBps": round(
-            nbytes / ms / 1e6, 1), "tokens_per_s": round(m * 1000.0 / ms, 1)}
+            nbytes / ms / 1e6, 1), "frac_of_hbm_measured": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
+            "tokens_per_s": round(m * 1000.0 / ms, 1)}
         del g, plan, probs
         torch.cuda.empty_cache()
     # prefill GEMM: gate/up 6912x2560 and down 2560x6912 at M = 512 and 2048
@@ -572,12 +947,8 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
                                    "frac_of_int8_peak": round(tops / int8_tops, 4),
                                    "frac_of_int8_spec_4500": round(tops / 4500.0, 4)}
             del g
-    pre["int8_peak_TOPS"] = round(int8_tops, 1)
-    pre["int8_peak_source"] = ("measured: torch._int_mm 8192^3 best of 10" if measured else
-                               f"{peaks['source']} bf16 burst x 2 (nominal int8/bf16 ratio)")
-    pre["int8_peak_derived_TOPS"] = round(derived, 1)
     out["prefill_gemm"] = pre
-    # single k_proj GEMV (640 x 2560, batch 1): one launch vs graph steady state
+    # single k_proj GEMV (640 x 2560, batch 1): one fused call, L2-resident
     w, _, _ = inputs.ternary_weights(640, 2560, inputs.seed_single())
     x = inputs.activations(1, 2560, inputs.seed_single())
     pr = Problem(i2s, torch, 640, 2560, 1, w, x.cuda(), torch.empty((1, 640), device="cuda"))
@@ -586,60 +957,34 @@ def extra_measurements(i2s, torch, inputs, steps: int, probs1, peaks):
     ms = time_replays(torch, g, 200, 10, collective=False)
     out["k_proj_single"] = {"us_per_call": round(ms * 1000, 2), "note": "L2-resident (0.41 MB)"}
     del g
-    # k_proj streamed: distinct copies of the packed tensor totalling more
-    # than 4x L2, one batched fused call per step
-    copies = int(4 * 126e6 / (640 * 2560 // 4)) + 1
-    xs_ = torch.empty((copies, 1, 2560), device="cuda").copy_(pr.x.view(1, 1, 2560).expand(copies, 1, 2560))
-    ys_ = torch.empty((copies, 1, 640), device="cuda")
-    pk = [pr.packed.clone() for _ in range(copies)]
-    plan = i2s.BatchedQuantGemv([(pk[i], 640, 2560, xs_[i], ys_[i], None) for i in range(copies)], 1)
-    g = capture(torch, plan.run)
-    ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
-    nbytes = copies * 640 * 2560 // 4
-    out["k_proj_streamed"] = {"copies": copies, "ms_per_step": round(ms, 4),
-                              "packed_GBps": round(nbytes / ms / 1e6, 1),
-                              "frac_of_hbm_measured": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
-    del g, plan, pk, xs_, ys_
-    torch.cuda.empty_cache()
-    # large BitNet-style layer (hidden 8192, ffn 28672): two device copies of
-    # its 7 projections (428 MB, more than 3x L2) at M = 1, and one at M = 64
-    large = inputs.projections_large()
-    packs = []
-    for idx, p in enumerate(large):
-        w = gpu_ternary(torch, p.n, p.k, inputs.seed_large(idx))
-        packs.append(i2s.bitnet_i2s_pack(w))
-        del w
-    torch.cuda.empty_cache()
-    layer_bytes = sum(p.n * p.k // 4 for p in large)
-    for m, ncopy in ((1, 2), (64, 1)):
-        probs, keep = [], []
-        for c in range(ncopy):
-            for idx, p in enumerate(large):
-                pk = packs[idx] if c == 0 else packs[idx].clone()
-                x = inputs.activations(m, p.k, inputs.seed_large(idx)).cuda()
-                y = torch.empty((m, p.n), device="cuda")
-                probs.append((pk, p.n, p.k, x, y, None))
-        plan = i2s.BatchedQuantGemv(probs, m)
-        g = capture(torch, plan.run)
-        ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
-        nbytes = ncopy * layer_bytes
-        ops = ncopy * sum(2.0 * m * p.n * p.k for p in large)
-        out[f"large_layer_M{m}"] = {
-            "layers": ncopy, "ms_per_step": round(ms, 4),
-            "packed_GBps": round(nbytes / ms / 1e6, 1),
-            "frac_of_hbm_measured": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
-            "TOPS": round(ops / ms / 1e9, 1), "frac_of_int8_peak": round(ops / ms / 1e9 / int8_tops, 4),
-            "tokens_per_s": round(m * 1000.0 / (ms / ncopy), 1)}
-        del g, plan, probs
+    # the other GEMV configs, one line each: 0 (k_proj streamed), 1 (one
+    # layer with outliers over 16 copies), 4 (large layer at M = 1 and 64)
+    for cfg, m in ((0, 1), (1, 1), (4, 1), (4, 64)):
+        wl = build_workload(i2s, torch, inputs, cfg, m, args.layers, 0)
+        gs = wl.graphs()
+        ms = time_replays(torch, gs, max(16, steps // 2), 3, collective=False)
+        key = {0: "k_proj_streamed", 1: "config1_layer_outliers", 4: f"large_layer_M{m}"}[cfg]
+        ent = {"ms_per_step": round(ms, 4), "packed_GBps": round(_packed(wl) / ms / 1e6, 1),
+               "frac_of_hbm_measured": round(_packed(wl) / ms / 1e6 / peaks["hbm_gbs"], 4),
+               "tokens_per_s": round(m * 1000.0 / ms, 1)}
+        if cfg == 4:
+            ops = sum(2.0 * m * p.n * p.k for p in wl.steps[0])
+            ent["TOPS"] = round(ops / ms / 1e9, 1)
+            ent["frac_of_int8_peak"] = round(ops / ms / 1e9 / int8_tops, 4)
+        out[key] = ent
+        del gs, wl
         torch.cuda.empty_cache()
-    del packs
-    torch.cuda.empty_cache()
     return out
+
+
+def _packed(wl) -> int:
+    return sum(p.packed_bytes for p in wl.steps[0])
 
 
 # ------------------------------------------------------------------- main
 
 def run_native(args):
+    import numpy as np
     import torch
 
     from i2_mpgemm_b200 import i2s, inputs
@@ -650,84 +995,106 @@ def run_native(args):
     dev = torch.device("cuda", local_rank)
     peaks = load_peaks()
     m = args.batch
-    if not 1 <= m <= 64:
-        raise SystemExit("--batch must be in 1..64")
+    cfg_id = args.config
+    if cfg_id != 3 and not 1 <= m <= 64:
+        raise SystemExit("--batch must be in 1..64 for the decode configs")
 
     # Each rank: a replica of the weights, its own activations.
-    stack = Stack(i2s, torch, inputs, args.layers, m, act_seed_offset=7919 * rank)
-    probs = stack.probs
-    packed_bytes = sum(p.packed_bytes for p in probs)
-    plan = stack_batch(i2s, probs)
-    dp4a = m <= 2
-    launches_per_step = step_launches(m, [p.k for p in probs])
-
-    g = capture(torch, plan.run)
+    work = build_workload(i2s, torch, inputs, cfg_id, m, args.layers, rank)
+    graphs = work.graphs()
     with ClockSampler(gpu_uuid(torch, local_rank)) as clk:
-        ms = time_replays(torch, g, args.steps, args.warmup)
+        ms = time_replays(torch, graphs, args.steps, args.warmup)
     ms = max_over_ranks(ms, dev)
     clocks = clk.summary()
-    value = world * packed_bytes / ms / 1e6  # GB/s over all ranks
+    scale = 1e6 if work.unit == "GB/s" else 1e9
+    value = world * work.work / ms / scale
 
-    # End to end through the public API: every step copies all 210 inputs
-    # from pinned host memory to the device (one copy), runs the step and
-    # copies all outputs back (one copy).
-    h2d = stack.x_dev.numel() * 4
-    d2h = stack.y_dev.numel() * 4
-    ms_e2e = time_replays(torch, g, args.steps, args.warmup, before=stack.h2d, after=stack.d2h)
+    # End to end through the public API: every step copies that step's
+    # inputs from pinned host memory to the device (one copy), runs the step
+    # and copies its outputs back (one copy).
+    h2d, d2h = work.io_bytes()
+    ms_e2e = time_replays(torch, graphs, args.steps, args.warmup, before=work.h2d, after=work.d2h)
     ms_e2e = max_over_ranks(ms_e2e, dev)
-    value_e2e = world * packed_bytes / ms_e2e / 1e6
+    value_e2e = world * work.work / ms_e2e / scale
 
     # Roofline of the dominant kernel (the matmul), per launch.
-    k_ms, k_launches, k_bytes = matmul_kernel_time(i2s, torch, probs)
-    achieved = k_bytes / (k_ms / 1000.0) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": measured_traffic() if dp4a else None, "peak_source": peaks["source"],
-                "kernel": ("i2s_gemv_dp4a_kernel (persistent launches of up to 160 problems)"
-                           if dp4a else "i2s_mma_kernel (persistent launches of up to 96 problems)"),
-                "launches_per_step": k_launches,
-                "bytes_per_launch": int(k_bytes // k_launches),
-                "launch_us_mean": round(1000 * k_ms / k_launches, 3)}
+    dp4a = all((m <= 2 and p.k <= 8192) or (m == 1 and p.k <= 30720) for p in work.steps[0])
+    if work.unit == "GB/s":
+        k_ms, k_launches, k_bytes = matmul_kernel_time(i2s, torch, work.steps)
+        achieved = k_bytes / (k_ms / 1000.0) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                    "traffic": measured_traffic() if (dp4a and cfg_id == 2 and m == 1) else None,
+                    "peak_source": peaks["source"],
+                    "kernel": ("i2s_gemv_dp4a_kernel (persistent launches of up to 160 problems)"
+                               if dp4a else
+                               "i2s_mma_kernel (persistent launches of up to 96 problems)"),
+                    "launches_per_step": k_launches,
+                    "bytes_per_launch": int(k_bytes // k_launches),
+                    "launch_us_mean": round(1000 * k_ms / k_launches, 3)}
+    else:
+        int8_tops, int8_src = int8_peak(torch, peaks)
+        k_ms, k_launches, _ = matmul_kernel_time(i2s, torch, work.steps)
+        achieved = work.work / (k_ms / 1000.0) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_tops, 1),
+                    "unit": "TOPS", "frac": round(achieved / int8_tops, 4), "traffic": None,
+                    "peak_source": int8_src,
+                    "kernel": "i2s_mma_kernel (persistent tcgen05 kind::i8)",
+                    "launches_per_step": k_launches,
+                    "ops_per_launch": int(work.work // k_launches),
+                    "launch_us_mean": round(1000 * k_ms / k_launches, 3)}
 
     # Secondary measurements: one process only (with more ranks the others
     # would wait at the final barrier longer than the process-group timeout),
     # and no collective inside.
     extra = {}
-    if rank == 0 and world == 1 and not args.no_extra:
-        extra = extra_measurements(i2s, torch, inputs, args.steps, probs, peaks)
-    extra["step_frac_of_hbm_peak"] = round(value / world / peaks["hbm_gbs"], 4)
-    extra["step_frac_of_hbm_spec_8tbs"] = round(value / world / 8000.0, 4)
-    extra["kernel_frac_of_hbm_spec_8tbs"] = round(achieved / 8000.0, 4)
+    if rank == 0 and world == 1 and not args.no_extra and cfg_id == 2 and m == 1:
+        extra = extra_measurements(i2s, torch, inputs, args, work, graphs[0], peaks)
+    if work.unit == "GB/s":
+        extra["step_frac_of_hbm_peak"] = round(value / world / peaks["hbm_gbs"], 4)
+        extra["step_frac_of_hbm_spec_8tbs"] = round(value / world / 8000.0, 4)
+        extra["kernel_frac_of_hbm_spec_8tbs"] = round(achieved / 8000.0, 4)
     extra["tokens_per_s"] = round(world * m * 1000.0 / ms, 1)
+    extra["tokens_per_s_note"] = ("independent problems in one call per step; "
+                                  "extra.stack_staged_* gives the dependency-staged step")
 
     cpu = None
     if rank == 0 and world == 1:
-        cpu = cpu_baseline(inputs, m, args.cpu_seconds)
-        if not args.no_extra:
+        # the outputs of the timed step for the problems the oracle sample
+        # runs (the first problems of step 0), for the parity check
+        n_sample = {0: 1, 1: 7, 2: 7, 3: 3, 4: 7}[cfg_id]
+        torch.cuda.synchronize()
+        work.plans[0].run()
+        torch.cuda.synchronize()
+        probs = work.steps[0]
+        if cfg_id == 3:
+            gpu_out = [p.y[:min(m, 4)].cpu().numpy() for p in probs[:n_sample]]
+        elif cfg_id == 4:
+            gpu_out = None  # device-drawn weights: the oracle sample draws its own on the host
+        else:
+            gpu_out = [p.y.cpu().numpy() for p in probs[:n_sample]]
+        cpu = cpu_baseline(inputs, cfg_id, m, args.cpu_seconds, gpu_out)
+        if not args.no_extra and cfg_id == 2:
             extra["cpu_baseline_all_cores"] = cpu_baseline_all_cores(m, args.cpu_seconds / 2)
 
-    cfg = workload_config(args.layers, m)
-    cfg["packed_bytes_per_step"] = packed_bytes
-    cfg["global_batch"] = m * world
-    cfg["parallelism"] = f"replicas x{world} (data parallel, no collective)"
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "metric": METRIC, "value": round(value, 1), "unit": work.unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded ternary weights p=.25/.5/.25 x U(0.5,2) scale, N(0,1) "
-                "activations)",
-        "config": cfg,
+        "data": DATA,
+        "config": workload_config(cfg_id, m, args.layers, world),
         "roofline": roofline,
         "cpu_baseline": cpu,
-        "e2e": {"value": round(value_e2e, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+        "parity_ok": None if cpu is None or "parity" not in cpu else cpu["parity"]["parity_ok"],
+        "e2e": {"value": round(value_e2e, 1), "unit": work.unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": work.launches * args.steps,
         "clocks": clocks,
         "extra": extra,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g
+    del graphs
     barrier()
     import torch.distributed as dist
     if dist.is_initialized():

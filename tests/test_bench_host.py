@@ -34,7 +34,7 @@ def test_launches_per_step(bench):
 
 
 def test_workload_config_counts_the_stack(bench):
-    cfg = bench.workload_config(30, 1)
+    cfg = bench.workload_config(2, 1, 30)
     n_k = [(2560, 2560), (640, 2560), (640, 2560), (2560, 2560), (6912, 2560), (6912, 2560),
            (2560, 6912)]
     assert cfg["packed_bytes_per_step"] == 30 * sum(n * k // 4 for n, k in n_k) == 521011200
@@ -61,3 +61,37 @@ def test_recorded_traffic_is_dropped_when_the_code_changes(bench, tmp_path, monk
         changed.append(str(dst))
     monkeypatch.setattr(bench, "DECODE_SOURCES", changed)
     assert bench.measured_traffic() is None
+
+
+def test_every_config_has_a_workload_and_the_reference_arm_prints_the_same_config(bench):
+    for c in range(5):
+        m = bench.DEFAULT_BATCH[c]
+        cfg = bench.workload_config(c, m, 30, 1)
+        assert cfg["workload"] and cfg["global_batch"] == m
+        assert cfg == bench.workload_config(c, m, 30, 1)
+    args = bench.parse_args(["--config", "3"])
+    assert args.batch == 2048
+    assert bench.parse_args([]).config == 2 and bench.parse_args([]).batch == 1
+
+
+def test_output_comparison_flags_a_wrong_or_nonzero_value(bench):
+    import numpy as np
+    want = [np.array([[1.0, 0.0, -2.0]], np.float32)]
+    assert bench.compare_outputs([want[0].copy()], want)["parity_ok"]
+    bad = want[0].copy()
+    bad[0, 2] = -2.001
+    assert not bench.compare_outputs([bad], want)["parity_ok"]
+    bad = want[0].copy()
+    bad[0, 1] = 1e-30
+    assert not bench.compare_outputs([bad], want)["parity_ok"]
+
+
+def test_reference_arm_line_on_a_small_sample(bench, capsys):
+    # config 0 at batch 1: one k_proj problem per step through the oracle
+    bench.run_reference(bench.parse_args(["--impl", "reference", "--config", "0", "--steps", "1",
+                                          "--warmup", "0"]))
+    import json
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["config"] == bench.workload_config(0, 1, 30, 1)
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
