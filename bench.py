@@ -957,6 +957,24 @@ def extra_measurements(i2s, torch, inputs, args, work, g_head, peaks):
     ms = time_replays(torch, g, 200, 10, collective=False)
     out["k_proj_single"] = {"us_per_call": round(ms * 1000, 2), "note": "L2-resident (0.41 MB)"}
     del g
+    # the block-64 IQ2_BN_R4 decode matmul at one token: four copies of a
+    # 28672 x 8192 weight (235 MB, over L2), one call each per step
+    n4, k4, copies = 28672, 8192, 4
+    w = gpu_ternary(torch, n4, k4, 40000)
+    r4s = [i2s.bitnet_iq2bn_pack(w, r4=True)]
+    del w
+    r4s += [r4s[0].clone() for _ in range(copies - 1)]
+    xq, xs = i2s.bitnet_act_quant_i8(inputs.activations(1, k4, 40000).cuda())
+    ys = [torch.empty((1, n4), device="cuda") for _ in range(copies)]
+    g = capture(torch, lambda: [i2s.bitnet_iq2bn_r4_gemv(r, n4, k4, xq, xs, y=y)
+                                for r, y in zip(r4s, ys)])
+    ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
+    nbytes = copies * n4 * k4 // 4
+    out["iq2bn_r4_gemv_M1"] = {"shape": f"{copies} x {n4}x{k4}", "ms_per_step": round(ms, 4),
+                               "packed_GBps": round(nbytes / ms / 1e6, 1),
+                               "frac_of_hbm_measured": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    del g, r4s, ys
+    torch.cuda.empty_cache()
     # the other GEMV configs, one line each: 0 (k_proj streamed), 1 (one
     # layer with outliers over 16 copies), 4 (large layer at M = 1 and 64)
     for cfg, m in ((0, 1), (1, 1), (4, 1), (4, 64)):

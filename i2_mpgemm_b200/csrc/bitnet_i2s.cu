@@ -334,7 +334,7 @@ bitnet_status plan_mma(MmaParamsT<CAP>& bp, const int8_t* const* xq) {
     if (st != BITNET_OK) return st;
     q.item_start = static_cast<int32_t>(items);
     q.chunk_start = static_cast<int32_t>(chunks);
-    const int64_t n_items = ((q.n + 127) / 128) * token_tiles;
+    const int64_t n_items = ((q.n + kMmaTileRows - 1) / kMmaTileRows) * token_tiles;
     items += n_items;
     chunks += n_items * ((q.k + 511) / 512);
     if (chunks > int64_t{0x7fffffff}) return fail(BITNET_ERR_SHAPE, "batch too large");
@@ -344,12 +344,12 @@ bitnet_status plan_mma(MmaParamsT<CAP>& bp, const int8_t* const* xq) {
   return BITNET_OK;
 }
 
-template <int T, bool kCodes, int CAP>
+template <int T, int CAP>
 bitnet_status launch_mma_t(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
                            bool pdl, bool wait, int dev) {
-  using C = MmaCfg<T, kCodes>;
+  using C = MmaCfg<T>;
   static std::atomic<uint8_t> smem_done[kMaxDevices];
-  auto kern = i2s_mma_kernel<T, kCodes, CAP>;
+  auto kern = i2s_mma_kernel<T, CAP>;
   bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
   if (st != BITNET_OK) return st;
   if ((st = plan_mma<T>(bp, xq)) != BITNET_OK) return st;
@@ -369,15 +369,15 @@ bitnet_status launch_mma_t(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStr
   return BITNET_OK;
 }
 
-// Token tile by M: small tiles with unsigned codes for decode, 128-token
-// tiles with signed weights for prefill.
+// Token tile by M: 16, 32 or 64 tokens for decode (3 or 4 CTAs per SM),
+// 128 for prefill (2 CTAs per SM).
 template <int CAP>
 bitnet_status launch_mma(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
                          bool pdl, bool wait, int dev) {
-  if (bp.m <= 16) return launch_mma_t<16, true>(bp, xq, stream, pdl, wait, dev);
-  if (bp.m <= 32) return launch_mma_t<32, true>(bp, xq, stream, pdl, wait, dev);
-  if (bp.m <= 64) return launch_mma_t<64, true>(bp, xq, stream, pdl, wait, dev);
-  return launch_mma_t<128, false>(bp, xq, stream, pdl, wait, dev);
+  if (bp.m <= 16) return launch_mma_t<16>(bp, xq, stream, pdl, wait, dev);
+  if (bp.m <= 32) return launch_mma_t<32>(bp, xq, stream, pdl, wait, dev);
+  if (bp.m <= 64) return launch_mma_t<64>(bp, xq, stream, pdl, wait, dev);
+  return launch_mma_t<128>(bp, xq, stream, pdl, wait, dev);
 }
 
 MmaProblem make_mma_problem(const uint8_t* packed, int64_t n, int64_t k, const float* xs, float* y,

@@ -10,10 +10,13 @@
 // Compared to Standard LLM Quantization", How I2_S Kernels Process the
 // Format) and contracted with the int8 activations.
 //
-// Tile ("swap-AB"): MMA M = 128 weight rows (operand A, held in TMEM), MMA
-// N = T tokens (operand B, Xq rows, K-major in shared memory), so a decode
-// batch of 3..64 tokens still fills the 128-row MMA.  A work item is one
-// 128 x T output tile over the whole K.  Items are numbered problem by
+// Tile ("swap-AB"): MMA M = 128 TMEM lanes (operand A), MMA N = T tokens
+// (operand B, Xq rows, K-major in shared memory), so a decode batch of 3..64
+// tokens still fills the 128-row MMA.  Lanes 0..126 hold 127 weight rows as
+// unsigned codes c = w + 1; lane 127 holds ones, so accumulator row 127 is
+// sum_k x for every token, and acc = D[r] - D[127] is the ternary
+// contraction of row r (w = c - 1).  A work item is one 127 x T output tile
+// over the whole K.  Items are numbered problem by
 // problem, token tile by token tile, row tile by row tile; each CTA owns one
 // contiguous range of items balanced by their 512-wide K chunks, and streams
 // through it without stopping between items.
@@ -26,11 +29,12 @@
 //   warp 1     TMEM allocator and MMA issuer (one thread).
 //   warps 2-5  unpack and epilogue: thread r (= TMEM lane r) owns weight row
 //              r of the tile.  Per block it expands its row's 32 bytes into 4
-//              groups x 32 int8 values and stores them as 32 TMEM columns (one
-//              A slot); a weight stage is released as soon as its bytes are in
-//              registers.  At the end of an item the same warps read the
-//              accumulator of their lane quarter and write y = ((float)acc *
-//              xs[m]) * s, token-major.
+//              groups x 32 codes and stores them as 32 TMEM columns (one A
+//              slot; lane 127 stores ones); a weight stage is released as soon
+//              as its bytes are in registers.  At the end of an item the same
+//              warps read the accumulator of their lane quarter and write
+//              y = ((float)acc * xs[m]) * s, token-major; the token sums of
+//              row 127 reach the other warps through shared memory.
 //
 // The MMA-issuing thread spends tens of cycles per small MMA, so a decode
 // tile keeps the tensor pipe fed only with several issuers per SM: small
@@ -40,19 +44,15 @@
 // Unpack: the 32-bit word made of bytes 4i..4i+3 of a block, shifted right
 // by 6-2g and masked with 0x03030303, is the four codes of weights
 // 32g+4i .. 32g+4i+3 in byte order, i.e. one TMEM column of the A operand
-// for the MMA over k = 32g .. 32g+31.  Two variants:
-//   kCodes = true:  A holds the unsigned codes c = w+1 (two ALU ops per four
-//     weights); the epilogue subtracts sum_k x, which the unpack warps add up
-//     from the activation boxes in shared memory.  For decode, where ALU
-//     issue is scarce and the MMAs are small.
-//   kCodes = false: A holds w itself (three more ALU ops per four weights).
-//     For prefill, where the unpack is amortised over 128 tokens.
+// for the MMA over k = 32g .. 32g+31: two ALU operations per four weights,
+// and no per-block work for the w = c - 1 correction, which the ones lane
+// does inside the MMA.
 //
 // Barriers: fullw/emptyw over the weight ring (TMA -> unpack), fullx/emptyx
-// over the activation ring (TMA -> MMA, and the unpack warps' token sums),
-// afull/aempty over the TMEM A slots (unpack -> MMA -> unpack), dfull/dempty
-// over the accumulator buffers (MMA -> epilogue -> MMA), xsum over the token
-// sums the unpack warps share.  Every wait is bounded (ptx.cuh); there are no
+// over the activation ring (TMA -> MMA), afull/aempty over the TMEM A slots
+// (unpack -> MMA -> unpack), dfull/dempty over the accumulator buffers
+// (MMA -> epilogue -> MMA), xsum over the token sums of row 127 (warp 3 ->
+// the other epilogue warps).  Every wait is bounded (ptx.cuh); there are no
 // named barriers, so a timed-out wait can never leave another warp stuck.
 #pragma once
 
@@ -90,7 +90,9 @@ struct MmaParamsT {
   MmaProblem p[CAP];
 };
 
-template <int T, bool kCodes>
+constexpr int kMmaTileRows = 127;  // weight rows per tile; TMEM lane 127 holds ones
+
+template <int T>
 struct MmaCfg {
   static_assert(T == 16 || T == 32 || T == 64 || T == 128, "token tile");
   static constexpr int kRows = 128;  // MMA M
@@ -111,18 +113,13 @@ struct MmaCfg {
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kWStages) * kWBytes +
                                        static_cast<size_t>(kXStages) * kXStageBytes +
                                        kNumBars * 8 + 2 * T * 4 + 16;
-  static constexpr uint32_t kIdesc = idesc_i8(128, T, !kCodes, true);
+  static constexpr uint32_t kIdesc = idesc_i8(128, T, false, true);  // u8 codes x s8
   static_assert(kTmemCols * kCtasPerSm <= 512, "tensor memory per SM");
   static_assert((kSmemBytes + 1024) * kCtasPerSm <= 228 * 1024, "shared memory per SM");
 };
 
-template <bool kCodes>
 __device__ __forceinline__ uint32_t unpack_word(uint32_t w, int g) {
-  const uint32_t c = (w >> (6 - 2 * g)) & 0x03030303u;
-  if (kCodes) return c;
-  // c in {0,1,2} per byte -> c - 1 per byte; the 0x80 bias keeps every byte
-  // from borrowing out of its neighbour.
-  return ((c | 0x80808080u) - 0x01010101u) ^ 0x80808080u;
+  return (w >> (6 - 2 * g)) & 0x03030303u;
 }
 
 template <typename BP>
@@ -159,16 +156,16 @@ template <typename BP>
 __device__ __forceinline__ void mma_item(const BP& bp, int item, int* p, int* rt, int* tt) {
   *p = mma_find_problem(bp, item);
   const MmaProblem& P = bp.p[*p];
-  const int row_tiles = (P.n + 127) >> 7;
+  const int row_tiles = (P.n + kMmaTileRows - 1) / kMmaTileRows;
   const int local = item - P.item_start;
   *tt = local / row_tiles;
   *rt = local - *tt * row_tiles;
 }
 
-template <int T, bool kCodes, int CAP>
-__global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
+template <int T, int CAP>
+__global__ void __launch_bounds__(192, MmaCfg<T>::kCtasPerSm)
     i2s_mma_kernel(const __grid_constant__ MmaParamsT<CAP> bp) {
-  using C = MmaCfg<T, kCodes>;
+  using C = MmaCfg<T>;
   constexpr int WS = C::kWStages, XS = C::kXStages, AS = C::kASlots, DB = C::kDBufs;
   constexpr int XB = C::kXB;
 
@@ -204,7 +201,7 @@ __global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
     }
     for (int s = 0; s < XS; ++s) {
       mbar_init(fullx_bar(s), 1);
-      mbar_init(emptyx_bar(s), kCodes ? 1 + 4 : 1);  // MMA commit (+ the token sums' reads)
+      mbar_init(emptyx_bar(s), 1);  // MMA commit
     }
     for (int t = 0; t < AS; ++t) {
       mbar_init(afull_bar(t), 4);
@@ -214,8 +211,8 @@ __global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
       mbar_init(dfull_bar(b), 1);
       mbar_init(dempty_bar(b), 4);
     }
-    mbar_init(xsum_bar(0), 4);
-    mbar_init(xsum_bar(1), 4);
+    mbar_init(xsum_bar(0), 1);  // lane 127's thread
+    mbar_init(xsum_bar(1), 1);
     misc[1] = 0u;
     fence_mbar_init();
   }
@@ -300,8 +297,8 @@ __global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
             }
           }
           mbar_arrive_expect_tx(fullw_bar(s), C::kWBytes);
-          tma_load_2d_hint(smem_u32(wring + s * C::kWBytes), &bp.tw[p], kc * 128, rt * 128,
-                           fullw_bar(s), pol_w);
+          tma_load_2d_hint(smem_u32(wring + s * C::kWBytes), &bp.tw[p], kc * 128,
+                           rt * kMmaTileRows, fullw_bar(s), pol_w);
           if (waited) {
             if (!issue_x(p, tt, kc)) {
               ok = false;
@@ -391,17 +388,13 @@ __global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const int ut = (warp - 2) * 32 + lane;  // 0..127 among the unpack warps
     bool ok = true;
-    int wc = 0, xc = 0, blk = 0, ii = 0;
+    int wc = 0, blk = 0, ii = 0;
     for (int item = item_lo; item < item_hi && ok; ++item, ++ii) {
       int p, rt, tt;
       mma_item(bp, item, &p, &rt, &tt);
       const MmaProblem& P = bp.p[p];
       const int nk = (P.k + 511) >> 9;
-      int xacc[T / 16];  // code mode: token sums over this thread's Xq chunks
-#pragma unroll
-      for (int i = 0; i < T / 16; ++i) xacc[i] = 0;
       for (int kc = 0; kc < nk && ok; ++kc, ++wc) {
         const int s = wc % WS;
         ok = __all_sync(0xffffffffu, mbar_wait(fullw_bar(s), (wc / WS) & 1, abort_flag));
@@ -411,40 +404,17 @@ __global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
         // then the stage goes back to the producer.  The box was written with
         // the 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r % 8).
         const uint8_t* wrow = wring + s * C::kWBytes + r * 128;
+        // Lane 127 carries ones: bytes of 0x55 unpack to code 1 in every group.
+        const uint4 ones = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
         uint4 wv4[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          wv4[c] = *reinterpret_cast<const uint4*>(wrow + ((c ^ (r & 7)) << 4));
+          wv4[c] = r == kMmaTileRows ? ones
+                                     : *reinterpret_cast<const uint4*>(wrow + ((c ^ (r & 7)) << 4));
         __syncwarp();
         if (lane == 0) mbar_arrive(emptyw_bar(s));
-        for (int q0 = 0; q0 < nb && ok; q0 += XB, ++xc) {
-          const int xs_ = xc % XS;
+        for (int q0 = 0; q0 < nb && ok; q0 += XB) {
           const int nbx = min(XB, nb - q0);
-          if (kCodes) {
-            // Token sums: each activation box holds T rows x 8 chunks of 16
-            // bytes; this thread adds chunk (ut % 8) of rows ut / 8 + 16 i.
-            // The swizzle only permutes chunks inside a row, so any chunk
-            // order will do.
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(fullx_bar(xs_), (xc / XS) & 1, abort_flag));
-            if (!ok) break;
-            const uint8_t* xst = xring + xs_ * C::kXStageBytes;
-            for (int q = 0; q < nbx; ++q) {
-#pragma unroll
-              for (int i = 0; i < T / 16; ++i) {
-                const uint4 v = *reinterpret_cast<const uint4*>(
-                    xst + q * C::kXBox + (ut / 8 + 16 * i) * 128 + (ut % 8) * 16);
-                int a = xacc[i];
-                a = __dp4a(static_cast<int>(v.x), 0x01010101, a);
-                a = __dp4a(static_cast<int>(v.y), 0x01010101, a);
-                a = __dp4a(static_cast<int>(v.z), 0x01010101, a);
-                a = __dp4a(static_cast<int>(v.w), 0x01010101, a);
-                xacc[i] = a;
-              }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(emptyx_bar(xs_));
-          }
           for (int q = 0; q < nbx; ++q, ++blk) {
             const int bi = q0 + q;  // block of the weight stage
             const uint4 c0 = wv4[2 * bi], c1 = wv4[2 * bi + 1];
@@ -453,7 +423,7 @@ __global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
 #pragma unroll
             for (int g = 0; g < 4; ++g)
 #pragma unroll
-              for (int i = 0; i < 8; ++i) a[8 * g + i] = unpack_word<kCodes>(wv[i], g);
+              for (int i = 0; i < 8; ++i) a[8 * g + i] = unpack_word(wv[i], g);
             const int t = blk % AS;
             if (blk >= AS) {
               // The slot's previous block has been read by its MMAs.
@@ -473,30 +443,31 @@ __global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
       if (!ok) break;
       // ---- epilogue of this item
       const int b = ii % DB;
-      if (kCodes) {
-        // Sum the 8 chunk threads of each token; share through shared memory.
-#pragma unroll
-        for (int i = 0; i < T / 16; ++i) {
-          int v = xacc[i];
-          v += __shfl_xor_sync(0xffffffffu, v, 1);
-          v += __shfl_xor_sync(0xffffffffu, v, 2);
-          v += __shfl_xor_sync(0xffffffffu, v, 4);
-          if ((ut & 7) == 0) xsum_smem[(ii & 1) * T + ut / 8 + 16 * i] = v;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(xsum_bar(ii & 1));
-      }
       ok = __all_sync(0xffffffffu, mbar_wait(dfull_bar(b), (ii / DB) & 1, abort_flag));
       if (!ok) break;
-      if (kCodes) {
-        ok = __all_sync(0xffffffffu, mbar_wait(xsum_bar(ii & 1), (ii >> 1) & 1, abort_flag));
-        if (!ok) break;
-      }
       tc_fence_after();
+      int32_t* xsum_buf = xsum_smem + (ii & 1) * T;
+      if (quarter == 3) {
+        // Row 127 (this warp's lane 31) holds sum_k x of every token.
+#pragma unroll 1
+        for (int c0 = 0; c0 < T; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem + lane_base + b * C::kDCols + c0, v);
+          tmem_ld_wait();
+          if (lane == 31) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) xsum_buf[c0 + j] = static_cast<int32_t>(v[j]);
+          }
+        }
+        if (lane == 31) mbar_arrive(xsum_bar(ii & 1));
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(xsum_bar(ii & 1), (ii >> 1) & 1, abort_flag));
+      if (!ok) break;
       const float s = *reinterpret_cast<const float*>(P.packed + static_cast<int64_t>(P.n) * (P.k >> 2));
-      const int64_t n = static_cast<int64_t>(rt) * 128 + r;
+      const int64_t n = static_cast<int64_t>(rt) * kMmaTileRows + r;
       const int64_t tok0 = static_cast<int64_t>(tt) * T;
       const int64_t nn = P.n;
+      const bool row_ok = r < kMmaTileRows && n < nn;
       float* __restrict__ yb = P.y;
       int32_t* __restrict__ ab = P.acc;
       const float* __restrict__ xsb = P.xs;
@@ -510,13 +481,12 @@ __global__ void __launch_bounds__(192, MmaCfg<T, kCodes>::kCtasPerSm)
         uint32_t v[16];
         tmem_ld_32x32b_x16(tmem + lane_base + b * C::kDCols + c0, v);
         tmem_ld_wait();
-        if (n < nn) {
+        if (row_ok) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int64_t tok = tok0 + c0 + j;
             if (tok < m_tokens) {
-              int32_t a = static_cast<int32_t>(v[j]);
-              if (kCodes) a -= xsum_smem[(ii & 1) * T + c0 + j];
+              const int32_t a = static_cast<int32_t>(v[j]) - xsum_buf[c0 + j];
               yb[tok * nn + n] = __fmul_rn(__fmul_rn(__int2float_rn(a), xsv[j]), s);
               if (ab != nullptr) ab[tok * nn + n] = a;
             }
