@@ -180,25 +180,43 @@ constexpr int64_t kSplitItemsMax = 512;
 size_t split_cnt_ints() { return static_cast<size_t>(kSplitItemsMax) * 4; }
 size_t split_part_ints(int64_t mt) { return static_cast<size_t>(kSplitItemsMax) * 128 * mt; }
 
-// K slices for the problems of one decode launch on `grid` CTAs.  When the
-// launch has fewer 128-row tiles than CTAs, every problem's K range is cut
-// into up to ceil(grid / tiles) slices of whole 512-wide boxes, keeping the
-// launch's items within kSplitItemsMax, so that the launch has work for
-// every CTA.
+// K slices for the problems of one decode launch on `grid` CTAs.  A problem
+// longer than the variant's activation slot (`max_cps` boxes of 512) is cut
+// into slices that fit it.  When the launch has fewer 128-row tiles than
+// CTAs, every problem's K range is cut into up to ceil(grid / tiles) slices
+// of whole boxes, keeping the launch's items within kSplitItemsMax, so that
+// the launch has work for every CTA.
+int64_t slices_for(int64_t nk, int64_t want, int64_t max_cps) {
+  int64_t sp = std::max<int64_t>((nk + max_cps - 1) / max_cps, std::min(want, nk));
+  sp = std::max<int64_t>(sp, 1);
+  const int64_t cps = (nk + sp - 1) / sp;
+  return (nk + cps - 1) / cps;
+}
+
 template <int CAP>
-void plan_splits(BatchParamsT<CAP>& bp, int64_t grid) {
+void plan_splits(BatchParamsT<CAP>& bp, int64_t grid, int64_t max_cps) {
   int64_t tiles = 0;
   for (int i = 0; i < bp.count; ++i) tiles += (bp.p[i].n + kGemvTileRows - 1) / kGemvTileRows;
   int64_t want = 1;
   if (bp.split_base != nullptr && tiles < grid)
     want = std::min((grid + tiles - 1) / tiles, kSplitItemsMax / tiles);
+  // Slices forced by the slot size come on top: lower `want` until the
+  // launch's items fit the split area.
+  for (; want > 1; --want) {
+    int64_t items = 0;
+    for (int i = 0; i < bp.count; ++i) {
+      const int64_t nk = (bp.p[i].k + 511) / 512;
+      const int64_t sp = slices_for(nk, want, max_cps);
+      if (sp > 1) items += ((bp.p[i].n + kGemvTileRows - 1) / kGemvTileRows) * sp;
+    }
+    if (items <= kSplitItemsMax) break;
+  }
   int64_t part = 0, cnt = 0;
   for (int i = 0; i < bp.count; ++i) {
     BatchProblem& q = bp.p[i];
     const int64_t nk = (q.k + 511) / 512;
-    int64_t sp = std::max<int64_t>(1, std::min(want, nk));
+    const int64_t sp = slices_for(nk, want, max_cps);
     const int64_t cps = (nk + sp - 1) / sp;
-    sp = (nk + cps - 1) / cps;
     q.splits = static_cast<int32_t>(sp);
     q.cps = static_cast<int32_t>(cps);
     q.part_off = static_cast<int32_t>(part);
@@ -213,14 +231,14 @@ void plan_splits(BatchParamsT<CAP>& bp, int64_t grid) {
 
 // Tensor maps, work items and their stage counts for every problem.
 template <int CAP>
-bitnet_status plan_items(BatchParamsT<CAP>& bp, int64_t grid) {
+bitnet_status plan_items(BatchParamsT<CAP>& bp, int64_t grid, int64_t max_cps) {
   if (bp.queue != nullptr) {
     // Items are handed out in order: the longest ones (largest K) first, so
     // that the last items taken are short and the CTAs end together.
     std::stable_sort(bp.p, bp.p + bp.count,
                      [](const BatchProblem& a, const BatchProblem& b) { return a.k > b.k; });
   }
-  plan_splits(bp, grid);
+  plan_splits(bp, grid, max_cps);
   int64_t items = 0, stages = 0;
   for (int i = 0; i < bp.count; ++i) {
     BatchProblem& q = bp.p[i];
@@ -262,7 +280,7 @@ bitnet_status launch_dp4a_t(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl
   using C = GemvCfg<MT, KMAX>;
   static std::atomic<uint8_t> smem_done[kMaxDevices];
   auto kern = i2s_gemv_dp4a_kernel<MT, CAP, KMAX>;
-  bitnet_status st = plan_items(bp, int64_t{C::kCtasPerSm} * sm_count(dev));
+  bitnet_status st = plan_items(bp, int64_t{C::kCtasPerSm} * sm_count(dev), KMAX / 512);
   if (st != BITNET_OK) return st;
   const int grid = std::min(bp.total_items, C::kCtasPerSm * sm_count(dev));
   st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
@@ -285,13 +303,17 @@ bitnet_status launch_dp4a_t(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl
 // `pdl`: launch as a dependent of the preceding grid; `wait`: its CTAs wait
 // for that grid before reading activations (skipped only when the caller
 // knows the activations were complete before the preceding grid started).
+// `long_variant`: problems with K > 8192 run on the long-K variant; without
+// it they are cut into K slices on the standard one (which needs the split
+// area of a workspace).
 template <int CAP>
 bitnet_status launch_dp4a(BatchParamsT<CAP>& bp, cudaStream_t stream, bool pdl, int dev,
-                          bool wait = true) {
+                          bool wait = true, bool long_variant = true) {
   bp.pdl = (pdl && wait) ? 1 : 0;
   int kmax = 0;
   for (int i = 0; i < bp.count; ++i) kmax = std::max(kmax, bp.p[i].k);
-  if (bp.m == 1 && long_k(kmax)) return launch_dp4a_t<1, CAP, kGemvMaxKLong>(bp, stream, pdl, dev);
+  if (bp.m == 1 && long_k(kmax) && (long_variant || bp.split_base == nullptr))
+    return launch_dp4a_t<1, CAP, kGemvMaxKLong>(bp, stream, pdl, dev);
   if (bp.m == 1) return launch_dp4a_t<1, CAP>(bp, stream, pdl, dev);
   return launch_dp4a_t<2, CAP>(bp, stream, pdl, dev);
 }
@@ -505,17 +527,35 @@ DecodeTail decode_tail(void* base, int count, int64_t m) {
   return t;
 }
 
+// One decode launch: problems [lo, hi) of the index list, and its variant.
+struct DecodeChunk {
+  size_t lo, hi;
+  bool long_variant;  // K > 8192 on the long-K variant (else sliced)
+};
+
 // Cuts the decode problems (indices into a batch; `nk_of(i)` gives problem
 // i's N and K) into launches of at most kMaxBatch problems, in chunks of
-// equal size.  A launch runs one kernel variant, chosen by its largest K.
-// When the long-K problems have fewer 128-row tiles than the long-K variant
-// keeps CTAs on the GPU, every problem joins them in that variant, so the
-// launch still has work for every CTA; otherwise the two kinds get separate
-// launches.
+// equal size.  With a split area (`can_slice`), one-token problems with
+// K > 8192 run in K slices on the standard variant, as many as the split
+// area holds.  The others run on the long-K variant: when they have fewer
+// 128-row tiles than that variant keeps CTAs on the GPU, every problem
+// joins them there, so the launch still has work for every CTA; otherwise
+// the two kinds get separate launches.
 template <typename NKOf>
-std::vector<std::pair<size_t, size_t>> decode_chunks(std::vector<int>& idx, NKOf nk_of, int dev) {
-  const auto mid = std::stable_partition(idx.begin(), idx.end(),
-                                         [&](int i) { return !long_k(nk_of(i).second); });
+std::vector<DecodeChunk> decode_chunks(std::vector<int>& idx, NKOf nk_of, int dev,
+                                       bool can_slice) {
+  int64_t sliced_items = 0;
+  auto short_or_sliced = [&](int i) {
+    const auto nk = nk_of(i);
+    if (!long_k(nk.second)) return true;
+    if (!can_slice) return false;
+    const int64_t items = ((nk.first + kGemvTileRows - 1) / kGemvTileRows) *
+                          slices_for((nk.second + 511) / 512, 1, kGemvMaxK / 512);
+    if (sliced_items + items > kSplitItemsMax) return false;
+    sliced_items += items;
+    return true;
+  };
+  const auto mid = std::stable_partition(idx.begin(), idx.end(), short_or_sliced);
   size_t split = static_cast<size_t>(mid - idx.begin());
   int64_t long_tiles = 0;
   for (size_t j = split; j < idx.size(); ++j)
@@ -523,13 +563,14 @@ std::vector<std::pair<size_t, size_t>> decode_chunks(std::vector<int>& idx, NKOf
   const int64_t long_ctas =
       static_cast<int64_t>(GemvCfg<1, kGemvMaxKLong>::kCtasPerSm) * sm_count(dev);
   if (split < idx.size() && long_tiles < long_ctas) split = 0;  // one group
-  std::vector<std::pair<size_t, size_t>> out;
+  std::vector<DecodeChunk> out;
   for (const auto& g : {std::make_pair(size_t{0}, split), std::make_pair(split, idx.size())}) {
     const size_t n = g.second - g.first;
     if (n == 0) continue;
+    const bool long_variant = g.first == split || split == 0;
     const size_t nchunks = (n + kMaxBatch - 1) / kMaxBatch;
     for (size_t c = 0; c < nchunks; ++c)
-      out.emplace_back(g.first + n * c / nchunks, g.first + n * (c + 1) / nchunks);
+      out.push_back({g.first + n * c / nchunks, g.first + n * (c + 1) / nchunks, long_variant});
   }
   return out;
 }
@@ -602,10 +643,11 @@ bitnet_status run_quant_batched(const bitnet_i2s_problem* problems, int count, i
   bool first = true;
   if (!small.empty()) {
     const auto chunks = decode_chunks(
-        small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev);
+        small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev,
+        tail.part != nullptr);
     for (size_t c = 0; c < chunks.size(); ++c) {
-      const size_t lo = chunks[c].first;
-      const size_t hi = chunks[c].second;
+      const size_t lo = chunks[c].lo;
+      const size_t hi = chunks[c].hi;
       bp.count = static_cast<int32_t>(hi - lo);
       bp.m = static_cast<int32_t>(M);
       tail.assign(bp, c);
@@ -614,7 +656,8 @@ bitnet_status run_quant_batched(const bitnet_i2s_problem* problems, int count, i
         bp.p[i - lo] = make_problem(q.packed, q.N, q.K, sl[small[i]].first, sl[small[i]].second,
                                     q.Y, q.acc_or_null);
       }
-      bitnet_status st = launch_dp4a(bp, s, /*pdl=*/true, dev, /*wait=*/first);
+      bitnet_status st = launch_dp4a(bp, s, /*pdl=*/true, dev, /*wait=*/first,
+                                     chunks[c].long_variant);
       if (st != BITNET_OK) return st;
       first = false;
     }
@@ -894,7 +937,8 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
   bool first = true;
   if (!small.empty()) {
     const auto chunks = decode_chunks(
-        small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev);
+        small, [&](int i) { return std::make_pair(problems[i].N, problems[i].K); }, dev,
+        tail.part != nullptr);
     const size_t nchunks = chunks.size();
     if (workspace != nullptr) {
       // One grid zeroes the counters once the work before this call is done;
@@ -912,8 +956,8 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
       if (e != cudaSuccess) return cuda_fail(e, "launch of the counter reset");
     }
     for (size_t c = 0; c < nchunks; ++c) {
-      const size_t lo = chunks[c].first;
-      const size_t hi = chunks[c].second;
+      const size_t lo = chunks[c].lo;
+      const size_t hi = chunks[c].hi;
       bp.count = static_cast<int32_t>(hi - lo);
       bp.m = static_cast<int32_t>(M);
       tail.assign(bp, c);
@@ -922,7 +966,8 @@ bitnet_status bitnet_i2s_gemv_batched(const bitnet_i2s_qproblem* problems, int c
         bp.p[i - lo] = make_problem(q.packed, q.N, q.K, q.Xq, q.xs, q.Y, q.acc_or_null);
       }
       const bool after_reset = workspace != nullptr && c == 0;
-      st = launch_dp4a(bp, s, /*pdl=*/!first || after_reset, dev, /*wait=*/after_reset);
+      st = launch_dp4a(bp, s, /*pdl=*/!first || after_reset, dev, /*wait=*/after_reset,
+                       chunks[c].long_variant);
       if (st != BITNET_OK) return st;
       first = false;
     }

@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
       int issued = 0;    // boxes issued
       int nsw = 0;       // problem switches announced to the consumers
       int x_loaded = 0;  // switches whose activations were requested
-      int prev_p = -1;
+      int prev_p = -1, prev_sl = -1;
       bool waited = (bp.pdl == 0);
       if (waited) grid_dependents_launch();
       // Items: first this CTA's fixed range, then, with a work queue, items
@@ -252,6 +252,7 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
       // activations the next CTAs read stay there.
       const uint64_t pol_w = l2_policy_evict_first();
       int sw_problem[2] = {-1, -1};  // problem of each switch not yet loaded
+      int sw_klo[2] = {0, 0};        // first activation of its slot (K slices)
       bool ok = true;
       // Request the activations (and scales) of switch `j` into slot j & 1.
       auto load_x = [&](int j) -> bool {
@@ -262,9 +263,19 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
             *reinterpret_cast<const float*>(P.packed + static_cast<size_t>(P.n) * (P.k >> 2));
 #pragma unroll
         for (int m = 0; m < MT; ++m) xscal[4 * slot + 1 + m] = (m < m_tokens) ? P.xs[m] : 0.0f;
-        const uint32_t xbytes = static_cast<uint32_t>(m_tokens) * static_cast<uint32_t>(P.k);
-        mbar_arrive_expect_tx(xfull_bar(slot), xbytes);  // publishes xscal[slot]
-        bulk_load(smem_u32(xslots + slot * C::kXSlotBytes), P.xq, xbytes, xfull_bar(slot));
+        if (P.k <= KMAX) {
+          const uint32_t xbytes = static_cast<uint32_t>(m_tokens) * static_cast<uint32_t>(P.k);
+          mbar_arrive_expect_tx(xfull_bar(slot), xbytes);  // publishes xscal[slot]
+          bulk_load(smem_u32(xslots + slot * C::kXSlotBytes), P.xq, xbytes, xfull_bar(slot));
+        } else {
+          // A K slice: each token's activations k_lo .. k_hi, one after the other.
+          const int k_lo = sw_klo[slot];
+          const uint32_t len = static_cast<uint32_t>(min(P.k, k_lo + P.cps * 512) - k_lo);
+          mbar_arrive_expect_tx(xfull_bar(slot), static_cast<uint32_t>(m_tokens) * len);
+          for (int m = 0; m < m_tokens; ++m)
+            bulk_load(smem_u32(xslots + slot * C::kXSlotBytes + m * len),
+                      P.xq + static_cast<int64_t>(m) * P.k + k_lo, len, xfull_bar(slot));
+        }
         return true;
       };
       auto load_pending_x = [&]() {
@@ -309,7 +320,8 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
             }
           }
           int info = (kc == kc_lo ? 1 : 0) | (kc == kc_hi - 1 ? 2 : 0);
-          if (kc == kc_lo && p != prev_p) {
+          // A new problem, or a new K slice of one too long for the slot.
+          if (kc == kc_lo && (p != prev_p || (P.k > KMAX && sl != prev_sl))) {
             // At most two switches wait for their activations: the slots.
             if (nsw - x_loaded >= 2) {
               if (!waited) wait_for_inputs();
@@ -318,9 +330,11 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
             }
             prefetch_tensormap(&bp.tmap[p]);
             sw_problem[nsw & 1] = p;
+            sw_klo[nsw & 1] = P.k > KMAX ? kc_lo * 512 : 0;
             info |= (nsw + 1) << 8;
             ++nsw;
             prev_p = p;
+            prev_sl = sl;
           }
           StageMeta md;
           md.p = p;
@@ -400,6 +414,7 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
   const uint8_t* xsm = xslots;
   int cur_slot = -1;
   int k = 0, n = 0, splits = 1;
+  int xoff = 0, xstride = 0;  // the slot holds activations xoff .. xoff + xstride of each token
   int kc_first = 0;  // first box of the current item
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
@@ -439,6 +454,8 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
       k = bp.p[md.p].k;
       n = bp.p[md.p].n;
       splits = bp.p[md.p].splits;
+      xoff = k > KMAX ? md.kc * 512 : 0;
+      xstride = k > KMAX ? min(k, xoff + bp.p[md.p].cps * 512) - xoff : k;
       wscale = xscal[4 * slot];
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
@@ -446,7 +463,7 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
         int sum = 0;
         if (m < m_tokens && splits == 1) {
           for (int off = lane * 16; off < k; off += 512) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xsm + m * k + off);
+            const uint4 v = *reinterpret_cast<const uint4*>(xsm + m * xstride + off);
             sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
             sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
             sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
@@ -473,7 +490,7 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
           int sum = 0;
           if (m < m_tokens) {
             for (int off = k_lo + lane * 16; off < k_hi; off += 512) {
-              const uint4 v = *reinterpret_cast<const uint4*>(xsm + m * k + off);
+              const uint4 v = *reinterpret_cast<const uint4*>(xsm + m * xstride + (off - xoff));
               sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
               sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
               sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
@@ -493,7 +510,7 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
       for (int m = 0; m < MT; ++m)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint8_t* xg = xsm + m * k + kblk + 32 * ((j + cp) & 3);
+          const uint8_t* xg = xsm + m * xstride + (kblk - xoff) + 32 * ((j + cp) & 3);
           const uint4 lo = *reinterpret_cast<const uint4*>(xg);
           const uint4 hi = *reinterpret_cast<const uint4*>(xg + 16);
           xr[m][j][0] = lo.x;

@@ -11,7 +11,11 @@ the C file lists the pages (by title and section) and every reading taken
 where they are silent.  Parity status: every function is pinned by the
 ``-m "not gpu"`` tests (worked example, closed forms, brute force, error
 bounds) except the AbsMean ternarization's choice of eps and tie rule, which
-the pages leave open.
+the pages leave open.  The block-64 formats (IQ2_BN, IQ2_BN_R4, IQ1_BN) are
+"parity unpinned" in their byte layout: the page elides the bits inside a
+block, so the layout is this oracle's reading; what the page and the
+arithmetic fix about them (sizes, block of 64, R4 as a 4-row permutation,
+lossless round trips, the trit decode, closed forms) is pinned.
 """
 from __future__ import annotations
 
