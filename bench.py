@@ -439,10 +439,14 @@ def oracle_layer_sample(inputs, m: int, outliers: bool = False, seed_fn=None):
     return sample
 
 
-def oracle_sample(inputs, config: int, m: int):
+def oracle_sample(inputs, config: int, m: int, w_large=None):
     """The bounded sample of a config's workload that the oracle runs: a list
     of (packed, n, k, x) problems, the unit of the rate, the work per pass
-    in that unit's base (bytes or int ops), and a description."""
+    in that unit's base (bytes or int ops), and a description.  For config 4
+    `w_large` is the down projection's fp32 ternary weights as the timed arm
+    drew them (seeded torch RNG on the device, copied to the host); the oracle
+    packs them itself.  Without it the host generator draws weights of the
+    same shape and distribution (timing only)."""
     import oracle
     if config == 0:
         w, _, _ = inputs.ternary_weights(640, 2560, inputs.seed_single())
@@ -467,7 +471,7 @@ def oracle_sample(inputs, config: int, m: int):
         return s, "TOPS", sum(2 * tok * n * k for _, n, k, _ in s), \
             f"the first {tok} of the {m} tokens through gate, up and down"
     p = inputs.projections_large()[6]  # down 8192 x 28672
-    w, _, _ = inputs.ternary_weights(p.n, p.k, inputs.seed_large(6))
+    w = w_large if w_large is not None else inputs.ternary_weights(p.n, p.k, inputs.seed_large(6))[0]
     x = inputs.activations(1, p.k, inputs.seed_large(6))
     return [(oracle.pack(w.numpy()), p.n, p.k, x.numpy())], "GB/s", p.n * p.k // 4, \
         "the large layer's down projection 8192x28672 at batch 1"
@@ -485,12 +489,12 @@ def rate(work: float, seconds: float, unit: str) -> float:
     return work / seconds / (1e9 if unit == "GB/s" else 1e12)
 
 
-def cpu_baseline(inputs, config: int, m: int, budget_s: float, gpu_outputs=None):
+def cpu_baseline(inputs, config: int, m: int, budget_s: float, gpu_outputs=None, w_large=None):
     """The oracle, one thread, on the config's bounded sample for about
     `budget_s`.  With `gpu_outputs` (the timed step's outputs of the same
     sample problems, host arrays), the first pass's outputs are compared
     with them at the tests' tolerance, and the verdict is reported."""
-    sample, unit, work, what = oracle_sample(inputs, config, m)
+    sample, unit, work, what = oracle_sample(inputs, config, m, w_large)
     done, spent, ys = 0, 0.0, None
     while spent < budget_s or done == 0:
         dt, out = oracle_pass(sample)
@@ -1093,13 +1097,19 @@ def run_native(args):
         work.plans[0].run()
         torch.cuda.synchronize()
         probs = work.steps[0]
+        w_large = None
         if cfg_id == 3:
             gpu_out = [p.y[:min(m, 4)].cpu().numpy() for p in probs[:n_sample]]
         elif cfg_id == 4:
-            gpu_out = None  # device-drawn weights: the oracle sample draws its own on the host
+            # the down projection of copy 0, on the weights the timed arm drew
+            pd = inputs.projections_large()[6]
+            gpu_out = [probs[6].y[:1].cpu().numpy()]
+            w_large = gpu_ternary(torch, pd.n, pd.k, inputs.seed_large(6)).cpu()
+            torch.cuda.empty_cache()
         else:
             gpu_out = [p.y.cpu().numpy() for p in probs[:n_sample]]
-        cpu = cpu_baseline(inputs, cfg_id, m, args.cpu_seconds, gpu_out)
+        cpu = cpu_baseline(inputs, cfg_id, m, args.cpu_seconds, gpu_out, w_large)
+        del w_large
         if not args.no_extra and cfg_id == 2:
             extra["cpu_baseline_all_cores"] = cpu_baseline_all_cores(m, args.cpu_seconds / 2)
 
