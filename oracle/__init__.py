@@ -271,3 +271,30 @@ def gemm_rows(t: np.ndarray, d: np.ndarray, xq: np.ndarray, xs: np.ndarray):
     _check(_load().i2s_oracle_gemm_rows(_p(t), _p(d), n, k, _p(xq), _p(xs), m, _p(y), _p(acc)),
            "gemm_rows")
     return y, acc
+
+
+def quant_gemm_chain(problems):
+    """A dependency chain of fused problems, run one after the other.
+
+    `problems` is a list in order; each entry is (packed, n, k, src) where
+    `src` is either an fp32 [m, k] array (an external input) or the index of
+    an earlier entry whose output Y [m, n_src] (n_src == k) is the input.
+    This is the seven projections of a BitNet b1.58 layer in a decode step
+    ("BitNet Inference Preprocessing: Converting Hugging Face Checkpoints to
+    I2S GGUF", The Two-Stage BitNet Inference Preprocessing Pipeline, names
+    them) where each quantizes its input per token before the ternary matmul
+    ("LLM Quantization Paradigms: FP8, AWQ, EXL2 & BitNet b1.58 in 2026",
+    section 5): nothing but quant_gemm applied in order, each on the fp32
+    output the one it reads has produced.  Returns [(Y, acc, xq, xs)]."""
+    out = []
+    for i, (packed, n, k, src) in enumerate(problems):
+        if isinstance(src, (int, np.integer)):
+            if not 0 <= src < i:
+                raise ValueError(f"problem {i} reads problem {src}, which does not come before it")
+            x = out[src][0]
+            if x.shape[1] != k:
+                raise ValueError(f"problem {i}: K={k} but its input has {x.shape[1]} columns")
+        else:
+            x = src
+        out.append(quant_gemm(packed, n, k, x))
+    return out
