@@ -824,50 +824,92 @@ def build_workload(i2s, torch, inputs, config: int, m: int, layers: int, rank: i
                     step_launches(m, [p.k for p in large] * copies))
 
 
-def staged_stack(i2s, torch, inputs, layers: int, m: int):
+def staged_problems(i2s, torch, inputs, layers: int, m: int):
     """A dependency-staged decode step over the stack's shapes: per layer
-    four ordered calls -- q+k+v on the layer input, o on q's output, gate+up
-    on o's output, down on gate's output, whose output is the next layer's
-    input -- 4 x layers batched fused calls, each stage reading what the one
-    before it wrote.  Weights are drawn on the device with a per-tensor scale
-    of 1/sqrt(K/2), so that the values passed from stage to stage keep their
-    size over 120 stages instead of overflowing; the matmul is the same.
-    Returns (list of BatchedQuantGemv in order, packed bytes per step)."""
+    four stages -- q+k+v on the layer input, o on q's output, gate+up on o's
+    output, down on gate's output, whose output is the next layer's input.
+    Weights are drawn on the device with a per-tensor scale of 1/sqrt(K/2),
+    so that the values passed from stage to stage keep their size over 120
+    stages instead of overflowing; the matmul is the same.  Returns
+    (problems as (packed, N, K, X, Y, None) in order, their stage numbers,
+    packed bytes, tensors to keep alive); a problem's X is the very tensor
+    an earlier problem writes as Y, or the external layer-0 input."""
     P = {p.name: p for p in inputs.projections_2b()}
-    keep, calls, nbytes = [], [], 0
+    keep, probs, stages, nbytes = [], [], [], 0
     h = torch.randn((m, P["q"].k), generator=torch.Generator(device="cuda").manual_seed(5),
                     device="cuda")
     keep.append(h)
     for layer in range(layers):
-        def proj(name, idx):
+        def add(name, idx, x, stage):
             p = P[name]
             w = gpu_ternary(torch, p.n, p.k, inputs.seed_stack(layer, idx),
                             scale=float((p.k / 2) ** -0.5))
             pk = i2s.bitnet_i2s_pack(w)
-            keep.append(pk)
-            return pk, p
-        def out(p):
             y = torch.empty((m, p.n), device="cuda")
-            keep.append(y)
+            keep.extend([pk, y])
+            probs.append((pk, p.n, p.k, x, y, None))
+            stages.append(stage)
             return y
-        (q, pq), (k_, pk_), (v, pv) = proj("q", 0), proj("k", 1), proj("v", 2)
-        yq, yk, yv = out(pq), out(pk_), out(pv)
-        calls.append(i2s.BatchedQuantGemv([(q, pq.n, pq.k, h, yq, None),
-                                           (k_, pk_.n, pk_.k, h, yk, None),
-                                           (v, pv.n, pv.k, h, yv, None)], m))
-        o, po = proj("o", 3)
-        yo = out(po)
-        calls.append(i2s.BatchedQuantGemv([(o, po.n, po.k, yq, yo, None)], m))
-        (g, pg), (u, pu) = proj("gate", 4), proj("up", 5)
-        yg, yu = out(pg), out(pu)
-        calls.append(i2s.BatchedQuantGemv([(g, pg.n, pg.k, yo, yg, None),
-                                           (u, pu.n, pu.k, yo, yu, None)], m))
-        d, pd = proj("down", 6)
-        h = out(pd)
-        calls.append(i2s.BatchedQuantGemv([(d, pd.n, pd.k, yg, h, None)], m))
+        st = 4 * layer
+        yq = add("q", 0, h, st)
+        add("k", 1, h, st)
+        add("v", 2, h, st)
+        yo = add("o", 3, yq, st + 1)
+        yg = add("gate", 4, yo, st + 2)
+        add("up", 5, yo, st + 2)
+        h = add("down", 6, yg, st + 3)
         nbytes += sum(n * k // 4 for n, k in STACK_SHAPES)
     torch.cuda.empty_cache()
+    return probs, stages, nbytes, keep
+
+
+def staged_stack(i2s, torch, inputs, layers: int, m: int, staged=None):
+    """The staged step as 4 x layers batched fused calls in order, each stage
+    reading what the one before it wrote.  Returns (list of BatchedQuantGemv
+    in order, packed bytes per step, tensors to keep alive)."""
+    probs, stages, nbytes, keep = staged or staged_problems(i2s, torch, inputs, layers, m)
+    calls = []
+    for st in range(stages[-1] + 1):
+        calls.append(i2s.BatchedQuantGemv([p for p, s in zip(probs, stages) if s == st], m))
     return calls, nbytes, keep
+
+
+def staged_chain(i2s, torch, inputs, layers: int, m: int, staged=None):
+    """The staged step as one bitnet_i2s_quant_gemv_chain call.  Returns
+    (QuantGemvChain, packed bytes per step, tensors to keep alive)."""
+    probs, stages, nbytes, keep = staged or staged_problems(i2s, torch, inputs, layers, m)
+    return i2s.QuantGemvChain(probs, stages, m), nbytes, keep
+
+
+def staged_chain_measurement(i2s, torch, inputs, layers, m, steps, peaks):
+    """The dependency-staged step as one chain call: its time, and whether
+    its outputs equal, bit for bit, those of the 4 x layers separate calls
+    on the same weights and input."""
+    staged = staged_problems(i2s, torch, inputs, layers, m)
+    calls, sbytes, keep = staged_stack(i2s, torch, inputs, layers, m, staged)
+    chain, _, _ = staged_chain(i2s, torch, inputs, layers, m, staged)
+    ys = [p[4] for p in staged[0]]
+    for c in calls:
+        c.run()
+    want = [y.clone() for y in ys]
+    for y in ys:
+        y.fill_(float("nan"))
+    chain.run()
+    torch.cuda.synchronize()
+    same = all(torch.equal(a, b) for a, b in zip(ys, want))
+    del want, calls
+    g = capture(torch, chain.run)
+    ms = time_replays(torch, g, max(5, steps // 2), 3, collective=False)
+    n = len(staged[0])
+    res = {"problems": n, "stages": staged[1][-1] + 1, "ms_per_step": round(ms, 4),
+           "packed_GBps": round(sbytes / ms / 1e6, 1),
+           "frac_of_hbm_measured": round(sbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
+           "tokens_per_s": round(m * 1000.0 / ms, 1),
+           "us_per_stage": round(1000.0 * ms / (staged[1][-1] + 1), 2),
+           "launches_per_step": 1 + -(-n // 128),
+           "matches_staged_calls": same}
+    del g, chain, keep, staged
+    return res
 
 
 def extra_measurements(i2s, torch, inputs, args, work, g_head, peaks):
@@ -920,6 +962,11 @@ def extra_measurements(i2s, torch, inputs, args, work, g_head, peaks):
             "tokens_per_s": round(m * 1000.0 / ms, 1),
             "launches_per_step": args.layers * sum(step_launches(m, ks) for ks in STAGE_KS)}
         del g, calls, keep
+        torch.cuda.empty_cache()
+    # the same dependency-staged step as one chain call (one or two tokens)
+    for m in (1, 2):
+        out[f"stack_staged_chain_batch{m}"] = staged_chain_measurement(
+            i2s, torch, inputs, args.layers, m, steps, peaks)
         torch.cuda.empty_cache()
     # the stack at batch 2, 4 and 16 (one batched call per step)
     for m in (2, 4, 16):

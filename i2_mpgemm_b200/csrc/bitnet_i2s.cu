@@ -11,11 +11,13 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <unordered_map>
 #include <utility>
 #include <vector>
 
 #include "bitnet_i2s.h"
 #include "bn_kernels.cuh"
+#include "chain_kernel.cuh"
 #include "gemv_kernel.cuh"
 #include "mma_kernel.cuh"
 #include "quant_kernels.cuh"
@@ -1202,6 +1204,245 @@ bitnet_status bitnet_iq2bn_r4_gemv(const uint8_t* packed, int64_t N, int64_t K, 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the IQ2_BN_R4 matmul kernel");
   return ok();
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ chains
+namespace {
+
+static_assert(sizeof(ChainParamsT<kChainBatch>) <= 32764, "chain kernel parameter block");
+
+// A checked chain: each problem's source and the workspace layout.
+//   int32 [0, launches)             work counters, one per launch
+//   int32 [done, done + count)      finished items per problem
+//   int32 [cnt, cnt + sum tiles)    finished slices per row tile
+//   int32 [acc, ...)                accumulators, M x N per problem (64-int aligned)
+//   ---- zero_bytes: all of the above is zeroed by the call ----
+//   fp32  [xs_off, + 2 * count)     activation scales per problem
+struct ChainPlan {
+  std::vector<int> src;
+  std::vector<int64_t> acc_off, cnt_off;
+  int64_t launches = 0, done = 0, cnt = 0, acc = 0;
+  size_t zero_bytes = 0, xs_off = 0, total_bytes = 0;
+};
+
+int64_t align64i(int64_t v) { return (v + 63) & ~int64_t{63}; }
+
+bitnet_status plan_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int count, int64_t M,
+                         ChainPlan* plan) {
+  const char* fn = "bitnet_i2s_quant_gemv_chain";
+  if (pr == nullptr || stage == nullptr || count < 1)
+    return fail(BITNET_ERR_INVALID_ARG, "%s: no problems", fn);
+  if (count > (1 << 20)) return fail(BITNET_ERR_SHAPE, "%s: %d problems", fn, count);
+  if (M < 1 || M > 2)
+    return fail(BITNET_ERR_SHAPE, "%s: M=%lld (one or two tokens)", fn, (long long)M);
+  for (int i = 0; i < count; ++i) {
+    const bitnet_i2s_problem& q = pr[i];
+    bitnet_status st = check_matmul_args(fn, q.packed, q.N, q.K, q.X, q.X, M, q.Y, 2);
+    if (st != BITNET_OK) return st;
+    if (q.acc_or_null != nullptr && !aligned(q.acc_or_null, 4))
+      return fail(BITNET_ERR_ALIGN, "%s: acc must be 4-byte aligned", fn);
+    const int32_t want = i == 0 ? 0 : stage[i - 1];
+    if (stage[i] != want && !(i > 0 && stage[i] == want + 1))
+      return fail(BITNET_ERR_INVALID_ARG,
+                  "%s: stage[%d]=%d: stages start at 0 and rise by 0 or 1 from problem to problem",
+                  fn, i, stage[i]);
+  }
+  // Outputs must not overlap one another.
+  std::vector<std::pair<uintptr_t, uintptr_t>> yr(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    const uintptr_t b = reinterpret_cast<uintptr_t>(pr[i].Y);
+    yr[i] = {b, b + static_cast<uintptr_t>(M * pr[i].N) * sizeof(float)};
+  }
+  std::sort(yr.begin(), yr.end());
+  for (size_t i = 1; i < yr.size(); ++i)
+    if (yr[i].first < yr[i - 1].second)
+      return fail(BITNET_ERR_INVALID_ARG, "%s: two problems' outputs overlap", fn);
+  // An input is either exactly an earlier stage's output (the same pointer,
+  // K equal to its N) or memory no output of the chain touches.
+  std::unordered_map<uintptr_t, int> by_y;
+  for (int i = 0; i < count; ++i) by_y[reinterpret_cast<uintptr_t>(pr[i].Y)] = i;
+  plan->src.assign(static_cast<size_t>(count), -1);
+  for (int i = 0; i < count; ++i) {
+    const uintptr_t xb = reinterpret_cast<uintptr_t>(pr[i].X);
+    const auto it = by_y.find(xb);
+    if (it != by_y.end()) {
+      const int j = it->second;
+      if (stage[j] >= stage[i])
+        return fail(BITNET_ERR_INVALID_ARG,
+                    "%s: problem %d reads the output of problem %d, which is not in an earlier "
+                    "stage", fn, i, j);
+      if (pr[j].N != pr[i].K)
+        return fail(BITNET_ERR_SHAPE, "%s: problem %d has K=%lld but reads an output of N=%lld",
+                    fn, i, (long long)pr[i].K, (long long)pr[j].N);
+      plan->src[i] = j;
+      continue;
+    }
+    const uintptr_t xe = xb + static_cast<uintptr_t>(M * pr[i].K) * sizeof(float);
+    // First output range that ends after the input starts.
+    auto hit = std::upper_bound(yr.begin(), yr.end(), std::make_pair(xb, ~uintptr_t{0}));
+    if (hit != yr.begin() && std::prev(hit)->second > xb) hit = std::prev(hit);
+    if (hit != yr.end() && hit->first < xe)
+      return fail(BITNET_ERR_INVALID_ARG,
+                  "%s: problem %d's input overlaps an output of the chain without being one", fn,
+                  i);
+  }
+  plan->launches = (count + kChainBatch - 1) / kChainBatch;
+  plan->done = plan->launches;
+  plan->cnt = plan->done + count;
+  int64_t off = plan->cnt;
+  plan->cnt_off.resize(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    plan->cnt_off[i] = off - plan->cnt;
+    off += (pr[i].N + kGemvTileRows - 1) / kGemvTileRows;
+  }
+  plan->acc = align64i(off);
+  off = 0;
+  plan->acc_off.resize(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    plan->acc_off[i] = off;
+    off += align64i(M * pr[i].N);
+  }
+  if (off > int64_t{0x7fffffff})
+    return fail(BITNET_ERR_SHAPE, "%s: too many outputs in one chain", fn);
+  plan->zero_bytes = align256(static_cast<size_t>(plan->acc + off) * sizeof(int32_t));
+  plan->xs_off = plan->zero_bytes;
+  plan->total_bytes = plan->xs_off + align256(static_cast<size_t>(count) * 2 * sizeof(float));
+  return BITNET_OK;
+}
+
+template <int MT>
+bitnet_status launch_chain_t(ChainParamsT<kChainBatch>& bp, cudaStream_t s, int dev) {
+  using C = ChainCfg<MT>;
+  static std::atomic<uint8_t> smem_done[kMaxDevices];
+  auto kern = i2s_chain_kernel<MT, kChainBatch>;
+  bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
+  if (st != BITNET_OK) return st;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min(bp.total_items, C::kCtasPerSm * sm_count(dev))));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr = pdl_attr(true);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, bp);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the I2_S chain kernel");
+  return BITNET_OK;
+}
+
+// K slices: each stage's problems are cut so that the stage has about as
+// many items as the grid has CTAs (at most 16 boxes, 8192 weights, per
+// slice); then a zeroing launch and the chain launches, at most kChainBatch
+// problems each.  Launch c + 1 starts its work only after launch c has
+// finished (its CTAs wait for the preceding grid first), so a problem may
+// read the output of one in an earlier launch.
+bitnet_status run_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int count, int64_t M,
+                        void* workspace, const ChainPlan& plan, cudaStream_t s, int dev) {
+  const int ctas = (M == 1 ? ChainCfg<1>::kCtasPerSm : ChainCfg<2>::kCtasPerSm) * sm_count(dev);
+  std::vector<int64_t> stage_tiles(static_cast<size_t>(stage[count - 1]) + 1, 0);
+  for (int i = 0; i < count; ++i)
+    stage_tiles[stage[i]] += (pr[i].N + kGemvTileRows - 1) / kGemvTileRows;
+  int32_t* w = static_cast<int32_t*>(workspace);
+  {
+    const int64_t n16 = static_cast<int64_t>(plan.zero_bytes / 16);
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(
+        std::max<int64_t>(1, std::min<int64_t>((n16 + 255) / 256, 2 * sm_count(dev)))));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr = pdl_attr(true);
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, chain_zero_kernel, reinterpret_cast<int4*>(w), n16);
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the chain zeroing kernel");
+  }
+  static thread_local ChainParamsT<kChainBatch> bp;  // 28 KB: kept off the stack
+  const int64_t nl = plan.launches;
+  std::vector<int32_t> items(static_cast<size_t>(count));
+  for (int64_t c = 0; c < nl; ++c) {
+    const int lo = static_cast<int>(count * c / nl);
+    const int hi = static_cast<int>(count * (c + 1) / nl);
+    bp.count = hi - lo;
+    bp.m = static_cast<int32_t>(M);
+    bp.queue = w + c;
+    bp.done = w + plan.done;
+    bp.cnt_base = w + plan.cnt;
+    bp.acc_base = w + plan.acc;
+    bp.xs_base = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + plan.xs_off);
+    int64_t item = 0;
+    for (int i = lo; i < hi; ++i) {
+      const bitnet_i2s_problem& q = pr[i];
+      ChainProblem& P = bp.p[i - lo];
+      const int64_t tiles = (q.N + kGemvTileRows - 1) / kGemvTileRows;
+      const int64_t nk = (q.K + 511) / 512;
+      const int64_t want = std::max<int64_t>(1, ctas / std::max<int64_t>(1, stage_tiles[stage[i]]));
+      const int64_t cps = std::min<int64_t>(kChainMaxCps, (nk + std::min(nk, want) - 1) / std::min(nk, want));
+      const int64_t splits = (nk + cps - 1) / cps;
+      bitnet_status st = encode_u8_2d(&bp.tmap[i - lo], q.packed, static_cast<uint64_t>(q.K / 4),
+                                      static_cast<uint64_t>(q.N), 128, kGemvTileRows);
+      if (st != BITNET_OK) return st;
+      const int j = plan.src[i];
+      P.packed = q.packed;
+      P.x = j < 0 ? q.X : nullptr;
+      P.src_scale = j < 0 ? nullptr
+                          : reinterpret_cast<const float*>(pr[j].packed + pr[j].N * (pr[j].K / 4));
+      P.y = q.Y;
+      P.acc_out = q.acc_or_null;
+      P.n = static_cast<int32_t>(q.N);
+      P.k = static_cast<int32_t>(q.K);
+      P.idx = i;
+      P.src = j;
+      P.src_items = j < 0 ? 0 : items[j];
+      P.src_acc = j < 0 ? 0 : static_cast<int32_t>(plan.acc_off[j]);
+      P.acc = static_cast<int32_t>(plan.acc_off[i]);
+      P.cnt = static_cast<int32_t>(plan.cnt_off[i]);
+      P.item_start = static_cast<int32_t>(item);
+      P.splits = static_cast<int32_t>(splits);
+      P.cps = static_cast<int32_t>(cps);
+      P.pad = 0;
+      items[i] = static_cast<int32_t>(tiles * splits);
+      item += tiles * splits;
+      if (item > int64_t{0x7fffffff}) return fail(BITNET_ERR_SHAPE, "chain too large");
+    }
+    bp.total_items = static_cast<int32_t>(item);
+    bp.pad = 0;
+    bitnet_status st = M == 1 ? launch_chain_t<1>(bp, s, dev) : launch_chain_t<2>(bp, s, dev);
+    if (st != BITNET_OK) return st;
+  }
+  return BITNET_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bitnet_i2s_quant_gemv_chain_workspace_bytes(const bitnet_i2s_problem* problems,
+                                                   const int32_t* stage, int count, int64_t M) {
+  ChainPlan plan;
+  return plan_chain(problems, stage, count, M, &plan) == BITNET_OK ? plan.total_bytes : 0;
+}
+
+bitnet_status bitnet_i2s_quant_gemv_chain(const bitnet_i2s_problem* problems, const int32_t* stage,
+                                          int count, int64_t M, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  ChainPlan plan;
+  bitnet_status st = plan_chain(problems, stage, count, M, &plan);
+  if (st != BITNET_OK) return st;
+  if (workspace == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_quant_gemv_chain: null workspace");
+  if (!aligned(workspace, 256))
+    return fail(BITNET_ERR_ALIGN, "bitnet_i2s_quant_gemv_chain: workspace must be 256-byte aligned");
+  if (workspace_bytes < plan.total_bytes)
+    return fail(BITNET_ERR_INVALID_ARG, "bitnet_i2s_quant_gemv_chain: workspace of %zu bytes < %zu",
+                workspace_bytes, plan.total_bytes);
+  int dev;
+  if ((st = check_device(&dev)) != BITNET_OK) return st;
+  st = run_chain(problems, stage, count, M, workspace, plan, static_cast<cudaStream_t>(stream), dev);
+  return st == BITNET_OK ? ok() : st;
 }
 
 }  // extern "C"

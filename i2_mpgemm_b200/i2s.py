@@ -43,6 +43,8 @@ SIGNATURES = {
     "bitnet_i2s_quant_gemv": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bitnet_i2s_quant_gemv_batched_workspace_bytes": (_SZ, [_VP, _I32, _I64]),
     "bitnet_i2s_quant_gemv_batched": (_I32, [_VP, _I32, _I64, _VP, _SZ, _VP]),
+    "bitnet_i2s_quant_gemv_chain_workspace_bytes": (_SZ, [_VP, _VP, _I32, _I64]),
+    "bitnet_i2s_quant_gemv_chain": (_I32, [_VP, _VP, _I32, _I64, _VP, _SZ, _VP]),
     "bitnet_i2s_gemv_batched_workspace_bytes": (_SZ, [_I32]),
     "bitnet_i2s_gemv_batched": (_I32, [_VP, _I32, _I64, _VP, _SZ, _VP]),
     "bitnet_i2s_quant_gemv_noalloc": (_I32, [_VP, _I64, _I64, _VP, _I64, _VP, _VP, _VP]),
@@ -284,6 +286,56 @@ class BatchedQuantGemv:
 def bitnet_i2s_quant_gemv_batched(problems, m: int, workspace=None, stream=None) -> None:
     """One call for many independent (packed, N, K, X, Y, acc) problems."""
     BatchedQuantGemv(problems, m, workspace).run(stream)
+
+
+class QuantGemvChain:
+    """Argument block of one bitnet_i2s_quant_gemv_chain call.
+
+    `problems` is a list of (packed, N, K, X, Y, acc_or_None) CUDA tensors
+    in dependency order and `stages` their stage numbers (0, then equal or
+    one more each time).  A problem whose X is the very tensor (same data
+    pointer) that an earlier stage's problem writes as Y reads that output;
+    every other X is an external input.  `run()` makes the call (capturable
+    in a CUDA graph)."""
+
+    def __init__(self, problems, stages, m: int, workspace: torch.Tensor | None = None):
+        self.m = int(m)
+        if len(stages) != len(problems):
+            raise ValueError("one stage number per problem")
+        self.tensors = []
+        arr = (Problem * len(problems))()
+        for i, (packed, n, k, x, y, acc) in enumerate(problems):
+            _need(packed, "packed", torch.uint8, bitnet_i2s_packed_bytes(n, k))
+            _need(x, "X", torch.float32, self.m * k)
+            _need(y, "Y", torch.float32, self.m * n)
+            if acc is not None:
+                _need(acc, "acc", torch.int32, self.m * n)
+            arr[i] = Problem(packed.data_ptr(), n, k, x.data_ptr(), y.data_ptr(),
+                             None if acc is None else acc.data_ptr())
+            self.tensors += [packed, x, y, acc]
+        self.array = arr
+        self.stages = (ctypes.c_int32 * len(stages))(*[int(v) for v in stages])
+        self.count = len(problems)
+        need = int(lib.bitnet_i2s_quant_gemv_chain_workspace_bytes(arr, self.stages, self.count,
+                                                                   self.m))
+        if need == 0:
+            raise BitnetError(1, (lib.bitnet_last_error() or b"invalid chain").decode())
+        self.device = problems[0][0].device
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+        _need(workspace, "workspace", torch.uint8, need)
+        for t in self.tensors + [workspace]:
+            _same_device(self.device, tensor=t)
+        self.workspace = workspace
+
+    def run(self, stream=None) -> None:
+        _run(self.device, lib.bitnet_i2s_quant_gemv_chain, self.array, self.stages, self.count,
+             self.m, self.workspace.data_ptr(), self.workspace.numel(), stream=stream)
+
+
+def bitnet_i2s_quant_gemv_chain(problems, stages, m: int, workspace=None, stream=None) -> None:
+    """One call for a dependency-ordered chain of (packed, N, K, X, Y, acc)."""
+    QuantGemvChain(problems, stages, m, workspace).run(stream)
 
 
 class QProblem(ctypes.Structure):

@@ -207,6 +207,46 @@ BITNET_API bitnet_status bitnet_i2s_quant_gemv_batched(const bitnet_i2s_problem*
                                                        int64_t M, void* workspace,
                                                        size_t workspace_bytes, void* stream);
 
+/* Workspace bytes bitnet_i2s_quant_gemv_chain needs (0 for bad arguments;
+ * the reason is then readable from bitnet_last_error()). */
+BITNET_API size_t bitnet_i2s_quant_gemv_chain_workspace_bytes(const bitnet_i2s_problem* problems,
+                                                              const int32_t* stage, int count,
+                                                              int64_t M);
+
+/* A chain of fused problems in dependency order, in one persistent launch
+ * per 128 problems (plus one that zeroes the workspace's counters): the
+ * same results as calling bitnet_i2s_quant_gemv_batched once per stage, in
+ * stage order, on the problems of that stage.  This is the shape of a
+ * decode step through a BitNet b1.58 layer, whose seven projections each
+ * quantize the output of one before them [P2, The Two-Stage BitNet Inference
+ * Preprocessing Pipeline: q, k, v, o, gate, up, down; P5 section 5: per-token
+ * AbsMax quantization before each ternary matmul].
+ *   problems: HOST array of `count` descriptors (read during the call only);
+ *     M = 1 or 2 tokens.
+ *   stage: HOST array of `count` stage numbers: stage[0] = 0, and each next
+ *     one equal to the one before it or one more.
+ *   A problem's X is either exactly the Y of a problem of an earlier stage
+ *     (the same pointer, K equal to that problem's N) -- it then reads that
+ *     output as the earlier call would have left it -- or memory that no
+ *     problem of the chain writes.  Outputs must not overlap one another;
+ *     anything else is BITNET_ERR_INVALID_ARG, checked before any launch.
+ *   The kernel never materialises a chained input in fp32: it quantizes
+ *     the earlier problem's exact int32 accumulators with that problem's
+ *     scales, in the order and rounding of the fp32 output, so the int8
+ *     activations, and with them every acc and Y, are bit-identical to
+ *     those of the stage-by-stage calls.
+ *   workspace: device scratch of at least
+ *     bitnet_i2s_quant_gemv_chain_workspace_bytes(problems, stage, count, M)
+ *     bytes, 256-byte aligned, not shared with work that may run at the same
+ *     time; its contents need not be initialised.
+ *   Dependencies are waited for on the device with bounded waits: a wait
+ *     that runs out (2 s) raises BITNET_ERR_DEVICE_TIMEOUT in
+ *     bitnet_device_status() and the launch ends early. */
+BITNET_API bitnet_status bitnet_i2s_quant_gemv_chain(const bitnet_i2s_problem* problems,
+                                                     const int32_t* stage, int count, int64_t M,
+                                                     void* workspace, size_t workspace_bytes,
+                                                     void* stream);
+
 /* One problem of bitnet_i2s_gemv_batched: activations already quantized. */
 typedef struct bitnet_i2s_qproblem {
   const uint8_t* packed;  /* I2_S tensor, 16-byte aligned */

@@ -163,3 +163,69 @@ def test_batched_workspace_layout(i2s):
     # the pre-quantized batched call sizes its split area for two tokens
     assert i2s.bitnet_i2s_gemv_batched_workspace_bytes(210) == (
         _align(4 * (launches + launches * 512 * 4)) + _align(4 * launches * 512 * 128 * 2))
+
+
+def _chain(i2s, specs, m):
+    """(descriptor array, stage array) of (N, K, X, Y, stage) fake-address specs."""
+    arr = (i2s.Problem * len(specs))()
+    stages = (ctypes.c_int32 * len(specs))()
+    for i, (n, k, x, y, st) in enumerate(specs):
+        arr[i] = i2s.Problem(A, n, k, x, y, None)
+        stages[i] = st
+    return arr, stages
+
+
+def _chain_bytes(i2s, specs, m):
+    arr, stages = _chain(i2s, specs, m)
+    return i2s.lib.bitnet_i2s_quant_gemv_chain_workspace_bytes(arr, stages, len(specs), m)
+
+
+def test_chain_workspace_layout(i2s):
+    """Work counters (one per launch of up to 128 problems), per-problem done
+    counters, per-row-tile counters, then M x N accumulators per problem
+    (64-int aligned): all zeroed; then two scales per problem."""
+    Y = 1 << 30  # outputs far apart
+    specs = [(2560, 2560, A, Y, 0), (640, 2560, A, Y + (1 << 24), 0),
+             (2560, 2560, Y, Y + (2 << 24), 1), (6912, 2560, Y + (2 << 24), Y + (3 << 24), 2),
+             (2560, 6912, Y + (3 << 24), Y + (4 << 24), 3)]
+    for m in (1, 2):
+        ints = 1 + len(specs) + sum(-(-n // 128) for n, *_ in specs)
+        ints = -(-ints // 64) * 64 + sum(-(-m * n // 64) * 64 for n, *_ in specs)
+        want = _align(4 * ints) + _align(8 * len(specs))
+        assert _chain_bytes(i2s, specs, m) == want, m
+    # 130 problems: two launches, two work counters
+    many = [(128, 128, A, Y + i * 4096, 0) for i in range(130)]
+    ints = 2 + 130 + 130
+    ints = -(-ints // 64) * 64 + 130 * 128
+    assert _chain_bytes(i2s, many, 1) == _align(4 * ints) + _align(8 * 130)
+
+
+def test_chain_argument_errors_on_host(i2s):
+    Y = 1 << 30
+    ok = [(256, 128, A, Y, 0), (128, 256, Y, Y + 4096, 1)]
+    assert _chain_bytes(i2s, ok, 1) > 0
+    bad = {
+        "three tokens": (ok, 3),
+        "stage not from 0": ([(256, 128, A, Y, 1)], 1),
+        "stage jumps": ([(256, 128, A, Y, 0), (128, 256, Y, Y + 4096, 2)], 1),
+        "stage falls": ([(256, 128, A, Y, 0), (128, 256, A, Y + 4096, 1),
+                         (128, 128, A, Y + 8192, 0)], 1),
+        "reads the same stage": ([(256, 128, A, Y, 0), (128, 256, Y, Y + 4096, 0)], 1),
+        "reads a later stage": ([(128, 256, Y, Y + 4096, 0), (256, 128, A, Y, 1)], 1),
+        "K differs from the source's N": ([(384, 128, A, Y, 0), (128, 256, Y, Y + 4096, 1)], 1),
+        "input inside an output": ([(256, 128, A, Y, 0), (128, 128, Y + 512, Y + 4096, 1)], 1),
+        "input straddles an output": ([(256, 128, A, Y + 512, 0), (128, 256, Y, Y + 8192, 1)], 1),
+        "outputs overlap": ([(256, 128, A, Y, 0), (256, 128, A, Y + 512, 0)], 1),
+        "unaligned input": ([(256, 128, A + 4, Y, 0)], 1),
+    }
+    for what, (specs, m) in bad.items():
+        assert _chain_bytes(i2s, specs, m) == 0, what
+        arr, stages = _chain(i2s, specs, m)
+        st = i2s.lib.bitnet_i2s_quant_gemv_chain(arr, stages, len(specs), m, A, 1 << 30, None)
+        assert st in (1, 2, 3), (what, st)
+    arr, stages = _chain(i2s, ok, 1)
+    need = _chain_bytes(i2s, ok, 1)
+    assert i2s.lib.bitnet_i2s_quant_gemv_chain(arr, stages, 2, 1, A, need - 1, None) == 1
+    assert i2s.lib.bitnet_i2s_quant_gemv_chain(arr, stages, 2, 1, A + 16, need, None) == 3
+    assert i2s.lib.bitnet_i2s_quant_gemv_chain(arr, stages, 2, 1, None, need, None) == 1
+    assert i2s.lib.bitnet_i2s_quant_gemv_chain(arr, None, 2, 1, A, need, None) == 1
