@@ -1214,8 +1214,7 @@ namespace {
 static_assert(sizeof(ChainParamsT<kChainBatch>) <= 32764, "chain kernel parameter block");
 
 // A checked chain: each problem's source and the workspace layout.
-//   int32 [0, launches)             work counters, one per launch
-//   int32 [done, done + count)      finished items per problem
+//   int32 [done, + 64 * count)      finished items per problem, 256 bytes apart
 //   int32 [cnt, cnt + sum tiles)    finished slices per row tile
 //   int32 [acc, ...)                accumulators, M x N per problem (64-int aligned)
 //   ---- zero_bytes: all of the above is zeroed by the call ----
@@ -1289,8 +1288,8 @@ bitnet_status plan_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int
                   i);
   }
   plan->launches = (count + kChainBatch - 1) / kChainBatch;
-  plan->done = plan->launches;
-  plan->cnt = plan->done + count;
+  plan->done = 0;
+  plan->cnt = plan->done + int64_t{count} * kChainDoneStride;
   int64_t off = plan->cnt;
   plan->cnt_off.resize(static_cast<size_t>(count));
   for (int i = 0; i < count; ++i) {
@@ -1312,23 +1311,47 @@ bitnet_status plan_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int
   return BITNET_OK;
 }
 
+// CTAs of the chain kernel that fit on the device at once.
 template <int MT>
-bitnet_status launch_chain_t(ChainParamsT<kChainBatch>& bp, cudaStream_t s, int dev) {
+bitnet_status chain_grid(int dev, int* out) {
   using C = ChainCfg<MT>;
   static std::atomic<uint8_t> smem_done[kMaxDevices];
+  static std::atomic<int> cached[kMaxDevices];
   auto kern = i2s_chain_kernel<MT, kChainBatch>;
   bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
   if (st != BITNET_OK) return st;
+  int v = cached[dev].load(std::memory_order_acquire);
+  if (v == 0) {
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads,
+                                                                  C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "occupancy of the I2_S chain kernel");
+    if (per_sm < 1) return fail(BITNET_ERR_UNSUPPORTED, "the chain kernel does not fit on an SM");
+    v = std::min(per_sm, C::kCtasPerSm) * sm_count(dev);
+    cached[dev].store(v, std::memory_order_release);
+  }
+  *out = v;
+  return BITNET_OK;
+}
+
+// A cooperative launch: all of its CTAs are resident at once, which the
+// kernel's fixed assignment of items to CTAs needs.
+template <int MT>
+bitnet_status launch_chain_t(ChainParamsT<kChainBatch>& bp, int grid, cudaStream_t s) {
+  using C = ChainCfg<MT>;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(static_cast<unsigned>(std::min(bp.total_items, C::kCtasPerSm * sm_count(dev))));
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min(bp.total_items, grid)));
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr = pdl_attr(true);
+  cudaLaunchAttribute attr;
+  std::memset(&attr, 0, sizeof(attr));
+  attr.id = cudaLaunchAttributeCooperative;
+  attr.val.cooperative = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, bp);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, i2s_chain_kernel<MT, kChainBatch>, bp);
   if (e != cudaSuccess) return cuda_fail(e, "launch of the I2_S chain kernel");
   return BITNET_OK;
 }
@@ -1336,12 +1359,13 @@ bitnet_status launch_chain_t(ChainParamsT<kChainBatch>& bp, cudaStream_t s, int 
 // K slices: each stage's problems are cut so that the stage has about as
 // many items as the grid has CTAs (at most 16 boxes, 8192 weights, per
 // slice); then a zeroing launch and the chain launches, at most kChainBatch
-// problems each.  Launch c + 1 starts its work only after launch c has
-// finished (its CTAs wait for the preceding grid first), so a problem may
-// read the output of one in an earlier launch.
+// problems each.  Launches follow one another in stream order, so a problem
+// may read the output of one in an earlier launch.
 bitnet_status run_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int count, int64_t M,
                         void* workspace, const ChainPlan& plan, cudaStream_t s, int dev) {
-  const int ctas = (M == 1 ? ChainCfg<1>::kCtasPerSm : ChainCfg<2>::kCtasPerSm) * sm_count(dev);
+  int ctas = 0;
+  bitnet_status gst = M == 1 ? chain_grid<1>(dev, &ctas) : chain_grid<2>(dev, &ctas);
+  if (gst != BITNET_OK) return gst;
   std::vector<int64_t> stage_tiles(static_cast<size_t>(stage[count - 1]) + 1, 0);
   for (int i = 0; i < count; ++i)
     stage_tiles[stage[i]] += (pr[i].N + kGemvTileRows - 1) / kGemvTileRows;
@@ -1354,9 +1378,6 @@ bitnet_status run_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int 
         std::max<int64_t>(1, std::min<int64_t>((n16 + 255) / 256, 2 * sm_count(dev)))));
     cfg.blockDim = dim3(256);
     cfg.stream = s;
-    cudaLaunchAttribute attr = pdl_attr(true);
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, chain_zero_kernel, reinterpret_cast<int4*>(w), n16);
     if (e != cudaSuccess) return cuda_fail(e, "launch of the chain zeroing kernel");
   }
@@ -1368,7 +1389,6 @@ bitnet_status run_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int 
     const int hi = static_cast<int>(count * (c + 1) / nl);
     bp.count = hi - lo;
     bp.m = static_cast<int32_t>(M);
-    bp.queue = w + c;
     bp.done = w + plan.done;
     bp.cnt_base = w + plan.cnt;
     bp.acc_base = w + plan.acc;
@@ -1410,7 +1430,7 @@ bitnet_status run_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int 
     }
     bp.total_items = static_cast<int32_t>(item);
     bp.pad = 0;
-    bitnet_status st = M == 1 ? launch_chain_t<1>(bp, s, dev) : launch_chain_t<2>(bp, s, dev);
+    bitnet_status st = M == 1 ? launch_chain_t<1>(bp, ctas, s) : launch_chain_t<2>(bp, ctas, s);
     if (st != BITNET_OK) return st;
   }
   return BITNET_OK;

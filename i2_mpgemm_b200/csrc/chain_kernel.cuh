@@ -16,11 +16,13 @@
 //   * A problem's input is either an external fp32 tensor or the output of
 //     one earlier problem (its `src`).  Problems come in dependency order.
 //   * Work item = (problem, K slice, row tile), numbered problem by problem;
-//     CTAs take items one at a time from a work counter, so an item is only
-//     ever taken after every item before it.  The producer warp streams the
-//     items' weight boxes (TMA, evict-first) into a ring: the weights do not
-//     depend on anything, so the ring fills with later items' weights while
-//     the compute warps wait for an earlier item's input.
+//     item i belongs to CTA i mod grid, and each CTA works through its items
+//     in increasing order.  A stage has at most about as many items as the
+//     grid has CTAs, so its items run on different CTAs side by side.  The
+//     producer warp streams the items' weight boxes (TMA, evict-first) into
+//     a ring: the weights do not depend on anything, so the ring fills with
+//     the CTA's next items' weights while the compute warps wait for an
+//     earlier item's input.
 //   * Item start: the compute warps wait (bounded) until every item of the
 //     source problem has finished (a per-problem counter in the workspace),
 //     take the token's absmax over the source's whole output, and quantize
@@ -39,11 +41,12 @@
 //     of a row tile writes the tile's fp32 outputs (and the optional int32
 //     copy) for the caller.
 //
-// Progress: an item waits only for items of an earlier problem, which were
-// all taken before it by CTAs already running; each CTA works through its
-// items in the order it took them.  So the lowest unfinished item never
-// waits on anything unfinished, and the chain always advances.  Every wait
-// is bounded all the same (device error flag, CTA abort).
+// Progress: an item waits only for items of earlier problems, which have
+// lower numbers; each CTA works through its items in increasing order, and
+// the launch is cooperative, so every CTA is resident.  So the lowest
+// unfinished item never waits on anything unfinished, and the chain always
+// advances.  Every wait is bounded all the same (device error flag, CTA
+// abort).
 //
 // The per-box arithmetic is the decode kernel's: mask-without-shift dp4a on
 // the 128-byte-swizzled box, four lanes per row, one I2_S block per lane.
@@ -55,6 +58,10 @@ namespace bitnet {
 
 constexpr int kChainMaxCps = 16;  // boxes per item at most: 8192 activations per token
 constexpr int kChainBatch = 128;  // problems per launch (parameter block under 32 KB)
+// Done counters sit 256 bytes apart: many CTAs poll them at once, and
+// counters sharing a line (and an L2 slice) would slow every poll and every
+// update of each other.
+constexpr int kChainDoneStride = 64;
 
 struct ChainProblem {
   const uint8_t* packed;   // I2_S tensor [n, k]
@@ -81,8 +88,7 @@ struct ChainParamsT {
   int32_t m;            // tokens
   int32_t total_items;  // work items of this launch
   int32_t pad;
-  int32_t* queue;       // this launch's work counter (zeroed)
-  int32_t* done;        // per chain problem: finished items (zeroed)
+  int32_t* done;        // per chain problem, kChainDoneStride ints apart: finished items (zeroed)
   int32_t* cnt_base;    // per row tile: finished slices (zeroed)
   int32_t* acc_base;    // int32 accumulators (zeroed)
   float* xs_base;       // per chain problem: two activation scales
@@ -110,23 +116,39 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
   return v;
 }
 
-// Bounded wait until *ctr >= target.  Gives up when `abort` is raised by
-// another thread of the CTA, or after kWaitTimeoutNs, raising `abort` and
-// the device error flag.
-__device__ __forceinline__ bool wait_count(const int32_t* ctr, int32_t target,
+__device__ __forceinline__ void red_release_gpu_add(int32_t* p, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t atom_acq_rel_gpu_add(int32_t* p, int32_t v) {
+  int32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Poll a counter (acquire loads at gpu scope) until *ctr >= target, then
+// publish `seq` in `seen`.  Gives up when `abort` is raised by another
+// thread of the CTA, or after kWaitTimeoutNs, raising `abort` and the device
+// error flag.  (Measured: back-off between polls, several staggered pollers
+// per CTA, or relaxed polls plus a fence change nothing or cost time.)
+__device__ __forceinline__ void poll_count(const int32_t* ctr, int32_t target, uint32_t delay_ns,
+                                           volatile uint32_t* seen, uint32_t seq,
                                            volatile uint32_t* abort) {
-  if (ld_acquire_gpu(ctr) >= target) return true;
+  if (delay_ns) __nanosleep(delay_ns);
   const uint64_t t0 = global_timer_ns();
-  while (true) {
-    for (int i = 0; i < 16; ++i) {
-      if (ld_acquire_gpu(ctr) >= target) return true;
-      __nanosleep(32);
+  for (int i = 0;; ++i) {
+    if (*seen == seq) return;
+    if (ld_acquire_gpu(ctr) >= target) {
+      *seen = seq;
+      return;
     }
-    if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-      *abort = 1u;
-      atomicOr(&g_error_flags, kErrWaitTimeout);
-      return false;
+    if ((i & 15) == 15) {
+      if (*abort) return;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        *abort = 1u;
+        atomicOr(&g_error_flags, kErrWaitTimeout);
+        return;
+      }
     }
   }
 }
@@ -157,6 +179,7 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
   uint32_t* red = reinterpret_cast<uint32_t*>(meta + S);  // [0,8): maxima, [8,16): sums
   volatile uint32_t* abort_flag = red + 16;
   volatile uint32_t* last_flag = red + 17;
+  volatile uint32_t* seen = red + 18;  // sequence number of the last item whose source was seen done
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -172,22 +195,24 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
     }
     mbar_init(cbar, C::kComputeWarps);
     *abort_flag = 0u;
+    *seen = 0u;
     fence_mbar_init();
   }
   __syncthreads();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // The work counter, and every input, come from earlier grids.
+    // The zeroed counters, and every input, come from earlier grids.
     grid_dependency_wait();
     grid_dependents_launch();
     if (lane != 0) return;
     const uint64_t pol_w = l2_policy_evict_first();
     int issued = 0;
     bool ok = true;
-    int item = atomicAdd(cp.queue, 1);
-    while (ok && item < cp.total_items) {
-      const int next = atomicAdd(cp.queue, 1);  // its result is used one item later
+    // Item i belongs to CTA i mod grid (the launch is cooperative: every
+    // CTA is resident), so the items of one stage run on different CTAs,
+    // side by side, and each CTA takes its items in increasing order.
+    for (int item = blockIdx.x; ok && item < cp.total_items; item += gridDim.x) {
       const int p = chain_problem_of(cp, item);
       const ChainProblem& P = cp.p[p];
       const int tiles = (P.n + kGemvTileRows - 1) / kGemvTileRows;
@@ -214,8 +239,8 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
                          full_bar(s), pol_w);
         ++issued;
       }
-      item = next;
     }
+    ok = ok && *abort_flag == 0u;
     if (ok) {
       // End of the work: a stage without data whose meta says so.
       const int s = issued % S;
@@ -253,11 +278,15 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
     gmask[j] = 0x03030303u << gshift[j];
   }
   uint32_t cphase = 0;
-  // All four compute warps meet; false when the CTA is aborting.
+  // All four compute warps meet; false when the CTA is aborting.  The
+  // second __syncwarp keeps the other lanes from probing the barrier before
+  // lane 0 has arrived: a diverged warp could otherwise spin on a phase that
+  // only its own lane 0, not yet scheduled, can complete.
   auto csync = [&]() -> bool {
     __syncwarp();
     if (lane == 0) mbar_arrive(cbar);
-    const bool ok = mbar_wait(cbar, cphase, abort_flag);
+    __syncwarp();
+    const bool ok = mbar_wait_spin(cbar, cphase, abort_flag);
     cphase ^= 1u;
     return __all_sync(0xffffffffu, ok) && *abort_flag == 0u;
   };
@@ -269,13 +298,16 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
   int xoff = 0, xstride = 0;
   // Absmax of the last input seen (source problem or external pointer).
   int cached_src = -2, cached_k = 0;
+  uint32_t nitem = 0;  // items begun (the same count in every compute thread)
   const float* cached_x = nullptr;
   float amax[MT];
+  float xs_in[MT];  // activation scales of the source problem
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     xsum[m] = 0;
     xsp[m] = 0.0f;
     amax[m] = 0.0f;
+    xs_in[m] = 0.0f;
   }
   int s = 0;
   uint32_t phase = 0;
@@ -298,76 +330,124 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
       const int k = P.k;
       const int k_lo = md.kc * 512;
       const int k_hi = min(k, k_lo + P.cps * 512);
+      const int nr = (k_hi - k_lo + 511) >> 9;  // 512-weight chunks in the slice
       xoff = k_lo;
-      xstride = min(P.cps, ((k + 511) >> 9) - md.kc) * 512;
+      xstride = nr * 512;
       wscale = __ldg(reinterpret_cast<const float*>(P.packed + static_cast<size_t>(P.n) * (k >> 2)));
       const bool chained = P.src >= 0;
-      if (chained && ctid == 0) wait_count(cp.done + P.src, P.src_items, abort_flag);
+      const float s_src = chained ? __ldg(P.src_scale) : 0.0f;
       const bool fresh = chained ? cached_src != P.src
                                  : (cached_src != -1 || cached_x != P.x || cached_k != k);
+      ++nitem;
+      // A source seen complete once stays complete: only a new one is waited for.
+      if (chained && fresh && ctid == 0)
+        poll_count(cp.done + P.src * kChainDoneStride, P.src_items, 0u, seen, nitem, abort_flag);
+      // The input row, as int4 words (int32 accumulators, or fp32 bits):
+      // thread ctid owns elements 4*ctid .. 4*ctid+3 of every 512-chunk.
+      const int4* src4 = chained ? reinterpret_cast<const int4*>(cp.acc_base + P.src_acc)
+                                 : reinterpret_cast<const int4*>(P.x);
+      // This thread's words of the slice's first two chunks, kept from the
+      // absmax pass so that slices of one or two chunks need no second read.
+      int4 keep[MT][2];
+      const bool kept = nr <= 2;
       if (fresh) {
         // Every thread waits here until the source is complete.
         if (!csync()) break;
+        // One load per CTA of the source's scales (every CTA of the stage
+        // reads the same word), shared through shared memory.
+        if (chained && ctid < MT) red[20 + ctid] = __float_as_uint(__ldcg(cp.xs_base + 2 * P.src + ctid));
+        // Eight 16-byte loads in flight per batch over all tokens' rows (one
+        // batch covers a 4096-wide row at one token).  Measured: more loads
+        // per batch (more registers) are slower at one and at two tokens.
+        constexpr int kB = 8 / MT;
+        // The CTAs of a stage all read the same row at once; each starts at
+        // its own chunk, so that they do not sweep its lines in step.
+        const int nch = (k + 511) >> 9;
+        const int rot = static_cast<int>(blockIdx.x % static_cast<unsigned>(nch));
+        uint32_t mx[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          uint32_t mx = 0;
-          if (chained) {
-            const int4* a4 = reinterpret_cast<const int4*>(cp.acc_base + P.src_acc +
-                                                           static_cast<int64_t>(m) * k);
-            for (int i = ctid; i < (k >> 2); i += 128) {
-              const int4 v = __ldcg(a4 + i);
-              mx = max(mx, max(max(static_cast<uint32_t>(abs(v.x)), static_cast<uint32_t>(abs(v.y))),
-                               max(static_cast<uint32_t>(abs(v.z)), static_cast<uint32_t>(abs(v.w)))));
+          mx[m] = 0;
+          keep[m][0] = make_int4(0, 0, 0, 0);
+          keep[m][1] = make_int4(0, 0, 0, 0);
+        }
+        for (int t0 = 0; t0 < nch; t0 += kB) {
+          int4 vb[MT][kB];
+#pragma unroll
+          for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+              const int r = t0 + u + rot < nch ? t0 + u + rot : t0 + u + rot - nch;
+              vb[m][u] = t0 + u < nch && r * 512 + 4 * ctid < k
+                             ? src4[static_cast<int64_t>(m) * (k >> 2) + r * 128 + ctid]
+                             : make_int4(0, 0, 0, 0);
             }
-          } else {
-            // Non-negative floats order like their bit patterns.
-            const float4* x4 =
-                reinterpret_cast<const float4*>(P.x + static_cast<int64_t>(m) * k);
-            for (int i = ctid; i < (k >> 2); i += 128) {
-              const float4 v = x4[i];
-              mx = max(mx, __float_as_uint(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)),
-                                                 fmaxf(fabsf(v.z), fabsf(v.w)))));
+#pragma unroll
+          for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+              const int r = t0 + u < nch ? (t0 + u + rot < nch ? t0 + u + rot : t0 + u + rot - nch)
+                                         : -1;
+              const int4 v = vb[m][u];
+              if (r == md.kc) keep[m][0] = v;
+              if (r == md.kc + 1) keep[m][1] = v;
+              if (chained) {
+                mx[m] = max(mx[m], max(max(static_cast<uint32_t>(abs(v.x)), static_cast<uint32_t>(abs(v.y))),
+                                       max(static_cast<uint32_t>(abs(v.z)), static_cast<uint32_t>(abs(v.w)))));
+              } else {
+                // Non-negative floats order like their bit patterns.
+                mx[m] = max(mx[m], max(max(static_cast<uint32_t>(v.x) & 0x7fffffffu,
+                                           static_cast<uint32_t>(v.y) & 0x7fffffffu),
+                                       max(static_cast<uint32_t>(v.z) & 0x7fffffffu,
+                                           static_cast<uint32_t>(v.w) & 0x7fffffffu)));
+              }
             }
-          }
-          mx = __reduce_max_sync(0xffffffffu, mx);
-          if (lane == 0) red[cw * 2 + m] = mx;
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const uint32_t w = __reduce_max_sync(0xffffffffu, mx[m]);
+          if (lane == 0) red[cw * 2 + m] = w;
         }
         if (!csync()) break;
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          uint32_t mx = max(max(red[m], red[2 + m]), max(red[4 + m], red[6 + m]));
-          if (chained) {
-            const float xs_src = __ldcg(cp.xs_base + 2 * P.src + m);
-            const float s_src = __ldg(P.src_scale);
-            amax[m] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(mx)), xs_src), s_src);
-          } else {
-            amax[m] = __uint_as_float(mx);
-          }
+          if (chained) xs_in[m] = __uint_as_float(red[20 + m]);
+          const uint32_t mx = max(max(red[m], red[2 + m]), max(red[4 + m], red[6 + m]));
+          amax[m] = chained
+                        ? __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(mx)), xs_in[m]), s_src)
+                        : __uint_as_float(mx);
         }
         cached_src = chained ? P.src : -1;
         cached_x = chained ? nullptr : P.x;
         cached_k = k;
+      } else if (kept) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const int4* row = src4 + static_cast<int64_t>(m) * (k >> 2);
+          keep[m][0] = k_lo + 4 * ctid < k_hi ? row[md.kc * 128 + ctid] : make_int4(0, 0, 0, 0);
+          keep[m][1] = k_lo + 512 + 4 * ctid < k_hi ? row[(md.kc + 1) * 128 + ctid]
+                                                     : make_int4(0, 0, 0, 0);
+        }
       }
       // Quantize the slice: q = clamp(rint(y * (127 / amax)), -127, 127),
       // and sum it for the unsigned-code correction.
-      const float s_src = chained ? __ldg(P.src_scale) : 0.0f;
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         const float inv = amax[m] > 0.0f ? __fdiv_rn(127.0f, amax[m]) : 0.0f;
         xsp[m] = amax[m] > 0.0f ? __fdiv_rn(amax[m], 127.0f) : 0.0f;
-        const float xs_src = chained ? __ldcg(cp.xs_base + 2 * P.src + m) : 0.0f;
+        const float xs_src = xs_in[m];
+        const int4* row = src4 + static_cast<int64_t>(m) * (k >> 2);
         int sum = 0;
-        for (int j = k_lo + 4 * ctid; j < k_hi; j += 512) {
+        auto quant4 = [&](int q, int4 raw) {
           float4 v;
           if (chained) {
-            const int4 q = __ldcg(reinterpret_cast<const int4*>(
-                cp.acc_base + P.src_acc + static_cast<int64_t>(m) * k + j));
-            v.x = __fmul_rn(__fmul_rn(__int2float_rn(q.x), xs_src), s_src);
-            v.y = __fmul_rn(__fmul_rn(__int2float_rn(q.y), xs_src), s_src);
-            v.z = __fmul_rn(__fmul_rn(__int2float_rn(q.z), xs_src), s_src);
-            v.w = __fmul_rn(__fmul_rn(__int2float_rn(q.w), xs_src), s_src);
+            v.x = __fmul_rn(__fmul_rn(__int2float_rn(raw.x), xs_src), s_src);
+            v.y = __fmul_rn(__fmul_rn(__int2float_rn(raw.y), xs_src), s_src);
+            v.z = __fmul_rn(__fmul_rn(__int2float_rn(raw.z), xs_src), s_src);
+            v.w = __fmul_rn(__fmul_rn(__int2float_rn(raw.w), xs_src), s_src);
           } else {
-            v = *reinterpret_cast<const float4*>(P.x + static_cast<int64_t>(m) * k + j);
+            v = make_float4(__int_as_float(raw.x), __int_as_float(raw.y), __int_as_float(raw.z),
+                            __int_as_float(raw.w));
           }
           const int q0 = max(-127, min(127, __float2int_rn(__fmul_rn(v.x, inv))));
           const int q1 = max(-127, min(127, __float2int_rn(__fmul_rn(v.y, inv))));
@@ -379,7 +459,14 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
           c.y = static_cast<signed char>(q1);
           c.z = static_cast<signed char>(q2);
           c.w = static_cast<signed char>(q3);
-          *reinterpret_cast<char4*>(xbuf + m * xstride + (j - k_lo)) = c;
+          *reinterpret_cast<char4*>(xbuf + m * xstride + q * 512 + 4 * ctid) = c;
+        };
+        if (kept) {
+          if (k_lo + 4 * ctid < k_hi) quant4(0, keep[m][0]);
+          if (k_lo + 512 + 4 * ctid < k_hi) quant4(1, keep[m][1]);
+        } else {
+          for (int q = 0; q < nr; ++q)
+            if (k_lo + q * 512 + 4 * ctid < k_hi) quant4(q, row[(md.kc + q) * 128 + ctid]);
         }
         sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0) red[8 + cw * 2 + m] = static_cast<uint32_t>(sum);
@@ -471,12 +558,14 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
           }
         }
       }
-      __threadfence();
+      // The barrier orders every thread's stores and adds before thread 0's
+      // release: the count makes them visible at gpu scope (cumulatively).
       if (!csync()) break;
       if (ctid == 0) {
-        atomicAdd(cp.done + P.idx, 1);
+        red_release_gpu_add(cp.done + P.idx * kChainDoneStride, 1);
         if (!whole)
-          *last_flag = atomicAdd(cp.cnt_base + P.cnt + md.row0 / kGemvTileRows, 1) == P.splits - 1;
+          *last_flag = atom_acq_rel_gpu_add(cp.cnt_base + P.cnt + md.row0 / kGemvTileRows, 1) ==
+                       P.splits - 1;
       }
       if (!whole) {
         if (!csync()) break;

@@ -96,6 +96,39 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait without suspending the thread: for short waits on the critical
+// path, where a parked thread's wake-up (about a microsecond) would cost more
+// than the issue slots the probing takes.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
+                                               volatile uint32_t* abort,
+                                               uint64_t timeout_ns = kWaitTimeoutNs) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (global_timer_ns() - t0 > timeout_ns) {
+      if (abort != nullptr) *abort = 1u;
+      atomicOr(&g_error_flags, kErrWaitTimeout);
+      return false;
+    }
+  }
+}
+
 // One bounded wait on an mbarrier that nothing ever completes: it runs out
 // after timeout_ns and raises the device error flag, exactly as a stuck
 // pipeline inside a real kernel would.  Used to test the reporting path.

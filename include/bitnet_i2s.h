@@ -213,8 +213,10 @@ BITNET_API size_t bitnet_i2s_quant_gemv_chain_workspace_bytes(const bitnet_i2s_p
                                                               const int32_t* stage, int count,
                                                               int64_t M);
 
-/* A chain of fused problems in dependency order, in one persistent launch
- * per 128 problems (plus one that zeroes the workspace's counters): the
+/* A chain of fused problems in dependency order, in one persistent
+ * cooperative launch per 128 problems (plus one that zeroes the workspace's
+ * counters; the cooperative launch needs every CTA of the grid resident, so
+ * the call fails with BITNET_ERR_CUDA where that cannot be had): the
  * same results as calling bitnet_i2s_quant_gemv_batched once per stage, in
  * stage order, on the problems of that stage.  This is the shape of a
  * decode step through a BitNet b1.58 layer, whose seven projections each

@@ -181,21 +181,21 @@ def _chain_bytes(i2s, specs, m):
 
 
 def test_chain_workspace_layout(i2s):
-    """Work counters (one per launch of up to 128 problems), per-problem done
-    counters, per-row-tile counters, then M x N accumulators per problem
-    (64-int aligned): all zeroed; then two scales per problem."""
+    """Per-problem done counters (256 bytes apart), per-row-tile counters, then M x N
+    accumulators per problem (64-int aligned): all zeroed; then two scales
+    per problem."""
     Y = 1 << 30  # outputs far apart
     specs = [(2560, 2560, A, Y, 0), (640, 2560, A, Y + (1 << 24), 0),
              (2560, 2560, Y, Y + (2 << 24), 1), (6912, 2560, Y + (2 << 24), Y + (3 << 24), 2),
              (2560, 6912, Y + (3 << 24), Y + (4 << 24), 3)]
     for m in (1, 2):
-        ints = 1 + len(specs) + sum(-(-n // 128) for n, *_ in specs)
+        ints = 64 * len(specs) + sum(-(-n // 128) for n, *_ in specs)
         ints = -(-ints // 64) * 64 + sum(-(-m * n // 64) * 64 for n, *_ in specs)
         want = _align(4 * ints) + _align(8 * len(specs))
         assert _chain_bytes(i2s, specs, m) == want, m
-    # 130 problems: two launches, two work counters
+    # 130 problems (two launches)
     many = [(128, 128, A, Y + i * 4096, 0) for i in range(130)]
-    ints = 2 + 130 + 130
+    ints = 64 * 130 + 130
     ints = -(-ints // 64) * 64 + 130 * 128
     assert _chain_bytes(i2s, many, 1) == _align(4 * ints) + _align(8 * 130)
 

@@ -191,7 +191,7 @@ def test_repeats_on_one_workspace_and_graph_replay(i2s):
             y.fill_(float("nan"))
         g.replay()
         ch.check(ref, "graph")
-    assert i2s.bitnet_device_status() == 0
+    i2s.bitnet_device_status()  # raises if a device-side wait ran out
 
 
 @pytest.mark.parametrize("m", [1, 2])
