@@ -1214,7 +1214,7 @@ namespace {
 static_assert(sizeof(ChainParamsT<kChainBatch>) <= 32764, "chain kernel parameter block");
 
 // A checked chain: each problem's source and the workspace layout.
-//   int32 [done, + 64 * count)      finished items per problem, 256 bytes apart
+//   int32 [0, 64 * count)           finished items per problem, 256 bytes apart
 //   int32 [cnt, cnt + sum tiles)    finished slices per row tile
 //   int32 [acc, ...)                accumulators, M x N per problem (64-int aligned)
 //   ---- zero_bytes: all of the above is zeroed by the call ----
@@ -1289,7 +1289,7 @@ bitnet_status plan_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int
   }
   plan->launches = (count + kChainBatch - 1) / kChainBatch;
   plan->done = 0;
-  plan->cnt = plan->done + int64_t{count} * kChainDoneStride;
+  plan->cnt = int64_t{count} * kChainDoneStride;
   int64_t off = plan->cnt;
   plan->cnt_off.resize(static_cast<size_t>(count));
   for (int i = 0; i < count; ++i) {
@@ -1383,7 +1383,7 @@ bitnet_status run_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int 
   }
   static thread_local ChainParamsT<kChainBatch> bp;  // 28 KB: kept off the stack
   const int64_t nl = plan.launches;
-  std::vector<int32_t> items(static_cast<size_t>(count));
+  std::vector<int32_t> splits_of(static_cast<size_t>(count)), items_of(static_cast<size_t>(count));
   for (int64_t c = 0; c < nl; ++c) {
     const int lo = static_cast<int>(count * c / nl);
     const int hi = static_cast<int>(count * (c + 1) / nl);
@@ -1416,15 +1416,17 @@ bitnet_status run_chain(const bitnet_i2s_problem* pr, const int32_t* stage, int 
       P.k = static_cast<int32_t>(q.K);
       P.idx = i;
       P.src = j;
-      P.src_items = j < 0 ? 0 : items[j];
+      P.src_splits = j < 0 ? 0 : splits_of[j];
+      P.src_cnt = j < 0 ? 0 : static_cast<int32_t>(plan.cnt_off[j]);
+      P.src_items = j < 0 ? 0 : items_of[j];
       P.src_acc = j < 0 ? 0 : static_cast<int32_t>(plan.acc_off[j]);
       P.acc = static_cast<int32_t>(plan.acc_off[i]);
       P.cnt = static_cast<int32_t>(plan.cnt_off[i]);
       P.item_start = static_cast<int32_t>(item);
       P.splits = static_cast<int32_t>(splits);
       P.cps = static_cast<int32_t>(cps);
-      P.pad = 0;
-      items[i] = static_cast<int32_t>(tiles * splits);
+      splits_of[i] = static_cast<int32_t>(splits);
+      items_of[i] = static_cast<int32_t>(tiles * splits);
       item += tiles * splits;
       if (item > int64_t{0x7fffffff}) return fail(BITNET_ERR_SHAPE, "chain too large");
     }

@@ -23,10 +23,10 @@
 //     a ring: the weights do not depend on anything, so the ring fills with
 //     the CTA's next items' weights while the compute warps wait for an
 //     earlier item's input.
-//   * Item start: the compute warps wait (bounded) until every item of the
-//     source problem has finished (a per-problem counter in the workspace),
-//     take the token's absmax over the source's whole output, and quantize
-//     just the item's K slice into shared memory.  The source's outputs are
+//   * Item start: the compute warps read the source problem's whole output,
+//     each 128-row tile as soon as its counter in the workspace says all of
+//     its K slices are in (bounded waits), take the token's absmax over it,
+//     and quantize just the item's K slice into shared memory.  The source's outputs are
 //     read as its exact int32 accumulators and turned into fp32 with the
 //     source's own scales, y = ((float)acc * xs) * s, the same operations
 //     and order as the output it writes, so every quantized value is the one
@@ -36,10 +36,10 @@
 //     the absmax of the output is y(max |acc|), exactly.
 //   * Item end: the slice's int32 row sums go to the problem's accumulators
 //     in the workspace (a plain store when the problem has one slice, an
-//     atomic add otherwise: integer sums are exact in any order); after a
-//     fence the item counts itself done.  The CTA that brings the last slice
-//     of a row tile writes the tile's fp32 outputs (and the optional int32
-//     copy) for the caller.
+//     atomic add otherwise: integer sums are exact in any order); then one
+//     release add counts the slice in its row tile's counter.  The CTA that
+//     brings the last slice of a row tile writes the tile's fp32 outputs (and
+//     the optional int32 copy) for the caller.
 //
 // Progress: an item waits only for items of earlier problems, which have
 // lower numbers; each CTA works through its items in increasing order, and
@@ -58,9 +58,8 @@ namespace bitnet {
 
 constexpr int kChainMaxCps = 16;  // boxes per item at most: 8192 activations per token
 constexpr int kChainBatch = 128;  // problems per launch (parameter block under 32 KB)
-// Done counters sit 256 bytes apart: many CTAs poll them at once, and
-// counters sharing a line (and an L2 slice) would slow every poll and every
-// update of each other.
+// One-token chains also count finished items per problem; these counters sit
+// 256 bytes apart, since all CTAs of a stage poll one of them at once.
 constexpr int kChainDoneStride = 64;
 
 struct ChainProblem {
@@ -70,16 +69,17 @@ struct ChainProblem {
   float* y;                // [m, n]
   int32_t* acc_out;        // [m, n] or null
   int32_t n, k;
-  int32_t idx;        // index in the whole chain: done counter and scale slot
+  int32_t idx;        // index in the whole chain: scale slot and done counter
   int32_t src;        // chain index of the problem whose output is the input, or -1
-  int32_t src_items;  // that problem's work items
+  int32_t src_splits; // that problem's K slices: a row tile of it is complete at this count
+  int32_t src_items;  // that problem's work items (all done: its output is complete)
+  int32_t src_cnt;    // its row-tile counters: cnt_base + src_cnt, [k / 128]
   int32_t src_acc;    // its accumulators: acc_base + src_acc, [m][k]
   int32_t acc;        // this problem's accumulators: acc_base + acc, [m][n]
   int32_t cnt;        // its row-tile arrival counters: cnt_base + cnt, [tiles]
   int32_t item_start; // first work item of this problem in its launch
   int32_t splits;     // K slices
   int32_t cps;        // boxes per slice (the last slice may have fewer)
-  int32_t pad;
 };
 
 template <int CAP>
@@ -126,28 +126,23 @@ __device__ __forceinline__ int32_t atom_acq_rel_gpu_add(int32_t* p, int32_t v) {
   return old;
 }
 
-// Poll a counter (acquire loads at gpu scope) until *ctr >= target, then
-// publish `seq` in `seen`.  Gives up when `abort` is raised by another
-// thread of the CTA, or after kWaitTimeoutNs, raising `abort` and the device
-// error flag.  (Measured: back-off between polls, several staggered pollers
-// per CTA, or relaxed polls plus a fence change nothing or cost time.)
-__device__ __forceinline__ void poll_count(const int32_t* ctr, int32_t target, uint32_t delay_ns,
-                                           volatile uint32_t* seen, uint32_t seq,
+// Bounded wait until *ctr >= target (acquire loads at gpu scope).  Gives
+// up when `abort` is raised by another thread of the CTA, or after
+// kWaitTimeoutNs, raising `abort` and the device error flag.  (Measured:
+// back-off between polls, several staggered pollers per CTA, or relaxed
+// polls plus a fence change nothing or cost time.)
+__device__ __forceinline__ bool wait_count(const int32_t* ctr, int32_t target,
                                            volatile uint32_t* abort) {
-  if (delay_ns) __nanosleep(delay_ns);
   const uint64_t t0 = global_timer_ns();
   for (int i = 0;; ++i) {
-    if (*seen == seq) return;
-    if (ld_acquire_gpu(ctr) >= target) {
-      *seen = seq;
-      return;
-    }
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    __nanosleep(32);
     if ((i & 15) == 15) {
-      if (*abort) return;
+      if (*abort) return false;
       if (global_timer_ns() - t0 > kWaitTimeoutNs) {
         *abort = 1u;
         atomicOr(&g_error_flags, kErrWaitTimeout);
-        return;
+        return false;
       }
     }
   }
@@ -179,7 +174,6 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
   uint32_t* red = reinterpret_cast<uint32_t*>(meta + S);  // [0,8): maxima, [8,16): sums
   volatile uint32_t* abort_flag = red + 16;
   volatile uint32_t* last_flag = red + 17;
-  volatile uint32_t* seen = red + 18;  // sequence number of the last item whose source was seen done
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -195,7 +189,6 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
     }
     mbar_init(cbar, C::kComputeWarps);
     *abort_flag = 0u;
-    *seen = 0u;
     fence_mbar_init();
   }
   __syncthreads();
@@ -298,7 +291,6 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
   int xoff = 0, xstride = 0;
   // Absmax of the last input seen (source problem or external pointer).
   int cached_src = -2, cached_k = 0;
-  uint32_t nitem = 0;  // items begun (the same count in every compute thread)
   const float* cached_x = nullptr;
   float amax[MT];
   float xs_in[MT];  // activation scales of the source problem
@@ -338,10 +330,6 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
       const float s_src = chained ? __ldg(P.src_scale) : 0.0f;
       const bool fresh = chained ? cached_src != P.src
                                  : (cached_src != -1 || cached_x != P.x || cached_k != k);
-      ++nitem;
-      // A source seen complete once stays complete: only a new one is waited for.
-      if (chained && fresh && ctid == 0)
-        poll_count(cp.done + P.src * kChainDoneStride, P.src_items, 0u, seen, nitem, abort_flag);
       // The input row, as int4 words (int32 accumulators, or fp32 bits):
       // thread ctid owns elements 4*ctid .. 4*ctid+3 of every 512-chunk.
       const int4* src4 = chained ? reinterpret_cast<const int4*>(cp.acc_base + P.src_acc)
@@ -350,20 +338,71 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
       // absmax pass so that slices of one or two chunks need no second read.
       int4 keep[MT][2];
       const bool kept = nr <= 2;
-      if (fresh) {
-        // Every thread waits here until the source is complete.
-        if (!csync()) break;
-        // One load per CTA of the source's scales (every CTA of the stage
-        // reads the same word), shared through shared memory.
-        if (chained && ctid < MT) red[20 + ctid] = __float_as_uint(__ldcg(cp.xs_base + 2 * P.src + ctid));
-        // Eight 16-byte loads in flight per batch over all tokens' rows (one
-        // batch covers a 4096-wide row at one token).  Measured: more loads
-        // per batch (more registers) are slower at one and at two tokens.
-        constexpr int kB = 8 / MT;
+      if (fresh && MT == 1) {
+        // One token: wait until every item of the source is done (one poller
+        // per CTA on the source's done counter), then read the whole row,
+        // eight 512-chunks per batch with their loads in flight together.
         // The CTAs of a stage all read the same row at once; each starts at
         // its own chunk, so that they do not sweep its lines in step.
+        if (chained && ctid == 0)
+          wait_count(cp.done + P.src * kChainDoneStride, P.src_items, abort_flag);
+        if (!csync()) break;
+        if (chained && ctid < MT)
+          red[20 + ctid] = __float_as_uint(__ldcg(cp.xs_base + 2 * P.src + ctid));
+        constexpr int kB = 8;
         const int nch = (k + 511) >> 9;
         const int rot = static_cast<int>(blockIdx.x % static_cast<unsigned>(nch));
+        uint32_t mx = 0;
+        keep[0][0] = make_int4(0, 0, 0, 0);
+        keep[0][1] = make_int4(0, 0, 0, 0);
+        for (int t0 = 0; t0 < nch; t0 += kB) {
+          int4 vb[kB];
+          int rr[kB];
+#pragma unroll
+          for (int u = 0; u < kB; ++u) {
+            const int r = t0 + u + rot < nch ? t0 + u + rot : t0 + u + rot - nch;
+            rr[u] = t0 + u < nch && r * 512 + 4 * ctid < k ? r : -1;
+            vb[u] = rr[u] >= 0 ? src4[rr[u] * 128 + ctid] : make_int4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int u = 0; u < kB; ++u) {
+            const int4 v = vb[u];
+            if (rr[u] == md.kc) keep[0][0] = v;
+            if (rr[u] >= 0 && rr[u] == md.kc + 1) keep[0][1] = v;
+            if (chained) {
+              mx = max(mx, max(max(static_cast<uint32_t>(abs(v.x)), static_cast<uint32_t>(abs(v.y))),
+                               max(static_cast<uint32_t>(abs(v.z)), static_cast<uint32_t>(abs(v.w)))));
+            } else {
+              // Non-negative floats order like their bit patterns.
+              mx = max(mx, max(max(static_cast<uint32_t>(v.x) & 0x7fffffffu,
+                                   static_cast<uint32_t>(v.y) & 0x7fffffffu),
+                               max(static_cast<uint32_t>(v.z) & 0x7fffffffu,
+                                   static_cast<uint32_t>(v.w) & 0x7fffffffu)));
+            }
+          }
+        }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) red[cw * 2] = mx;
+        if (!csync()) break;
+        if (chained) xs_in[0] = __uint_as_float(red[20]);
+        const uint32_t m0 = max(max(red[0], red[2]), max(red[4], red[6]));
+        amax[0] = chained ? __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(m0)), xs_in[0]), s_src)
+                          : __uint_as_float(m0);
+        cached_src = chained ? P.src : -1;
+        cached_x = chained ? nullptr : P.x;
+        cached_k = k;
+      } else if (fresh) {
+        // Two tokens: stream the source row in as its row tiles complete.  Chunk r (512
+        // values) holds row tiles 4r .. 4r+3; warp cw loads tile 4r + cw of
+        // every chunk, one 16-byte word per lane.  Lanes poll the tiles'
+        // counters in parallel (32 chunks per round) and the warp loads each
+        // tile as soon as it is seen complete, so that only the last tile's
+        // load is left after the source's last item finishes.  External
+        // inputs are loaded the same way without polls.
+        constexpr int kB = 8 / MT;  // chunks per load batch: eight loads in flight
+        const int nch = (k + 511) >> 9;
+        const int ntiles = k >> 7;
+        const int32_t* tcnt = chained ? cp.cnt_base + P.src_cnt : nullptr;
         uint32_t mx[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
@@ -371,43 +410,78 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
           keep[m][0] = make_int4(0, 0, 0, 0);
           keep[m][1] = make_int4(0, 0, 0, 0);
         }
-        for (int t0 = 0; t0 < nch; t0 += kB) {
-          int4 vb[MT][kB];
+        uint32_t xs_bits = 0;
+        bool waited = true;
+        for (int g0 = 0; g0 < nch && waited; g0 += 32) {
+          // Chunks g0 + i (i < 32) with a tile of this warp.
+          const int mine = min(32, (ntiles - cw + 3) / 4 - g0);
+          uint32_t pending = mine <= 0 ? 0u : (mine >= 32 ? 0xffffffffu : (1u << mine) - 1u);
+          const uint64_t t0 = global_timer_ns();
+          while (pending) {
+            bool ready = !chained;
+            if (chained && ((pending >> lane) & 1u))
+              ready = ld_acquire_gpu(tcnt + 4 * (g0 + lane) + cw) >= P.src_splits;
+            uint32_t fresh_tiles = __ballot_sync(0xffffffffu, ready) & pending;
+            __syncwarp();
+            // The first item of the source (tile 0) published its scales.
+            if (chained && cw == 0 && g0 == 0 && (fresh_tiles & 1u) && lane < MT)
+              xs_bits = __float_as_uint(__ldcg(cp.xs_base + 2 * P.src + lane));
+            pending &= ~fresh_tiles;
+            while (fresh_tiles) {
+              // Up to kB newly complete chunks per batch, loads in flight together.
+              int rr[kB];
 #pragma unroll
-          for (int m = 0; m < MT; ++m)
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-              const int r = t0 + u + rot < nch ? t0 + u + rot : t0 + u + rot - nch;
-              vb[m][u] = t0 + u < nch && r * 512 + 4 * ctid < k
-                             ? src4[static_cast<int64_t>(m) * (k >> 2) + r * 128 + ctid]
-                             : make_int4(0, 0, 0, 0);
-            }
-#pragma unroll
-          for (int m = 0; m < MT; ++m)
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-              const int r = t0 + u < nch ? (t0 + u + rot < nch ? t0 + u + rot : t0 + u + rot - nch)
-                                         : -1;
-              const int4 v = vb[m][u];
-              if (r == md.kc) keep[m][0] = v;
-              if (r == md.kc + 1) keep[m][1] = v;
-              if (chained) {
-                mx[m] = max(mx[m], max(max(static_cast<uint32_t>(abs(v.x)), static_cast<uint32_t>(abs(v.y))),
-                                       max(static_cast<uint32_t>(abs(v.z)), static_cast<uint32_t>(abs(v.w)))));
-              } else {
-                // Non-negative floats order like their bit patterns.
-                mx[m] = max(mx[m], max(max(static_cast<uint32_t>(v.x) & 0x7fffffffu,
-                                           static_cast<uint32_t>(v.y) & 0x7fffffffu),
-                                       max(static_cast<uint32_t>(v.z) & 0x7fffffffu,
-                                           static_cast<uint32_t>(v.w) & 0x7fffffffu)));
+              for (int u = 0; u < kB; ++u) {
+                rr[u] = fresh_tiles ? g0 + __ffs(fresh_tiles) - 1 : -1;
+                fresh_tiles &= fresh_tiles - 1;
               }
+              int4 vb[MT][kB];
+#pragma unroll
+              for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int u = 0; u < kB; ++u)
+                  vb[m][u] = rr[u] >= 0
+                                 ? src4[static_cast<int64_t>(m) * (k >> 2) + rr[u] * 128 + ctid]
+                                 : make_int4(0, 0, 0, 0);
+#pragma unroll
+              for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int u = 0; u < kB; ++u) {
+                  const int4 v = vb[m][u];
+                  if (rr[u] == md.kc) keep[m][0] = v;
+                  if (rr[u] >= 0 && rr[u] == md.kc + 1) keep[m][1] = v;
+                  if (chained) {
+                    mx[m] = max(mx[m], max(max(static_cast<uint32_t>(abs(v.x)), static_cast<uint32_t>(abs(v.y))),
+                                           max(static_cast<uint32_t>(abs(v.z)), static_cast<uint32_t>(abs(v.w)))));
+                  } else {
+                    // Non-negative floats order like their bit patterns.
+                    mx[m] = max(mx[m], max(max(static_cast<uint32_t>(v.x) & 0x7fffffffu,
+                                               static_cast<uint32_t>(v.y) & 0x7fffffffu),
+                                           max(static_cast<uint32_t>(v.z) & 0x7fffffffu,
+                                               static_cast<uint32_t>(v.w) & 0x7fffffffu)));
+                  }
+                }
             }
+            if (pending && global_timer_ns() - t0 > kWaitTimeoutNs) {
+              if (lane == 0) {
+                *abort_flag = 1u;
+                atomicOr(&g_error_flags, kErrWaitTimeout);
+              }
+              waited = false;
+              break;
+            }
+            if (pending && *abort_flag) {
+              waited = false;
+              break;
+            }
+          }
         }
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
           const uint32_t w = __reduce_max_sync(0xffffffffu, mx[m]);
           if (lane == 0) red[cw * 2 + m] = w;
         }
+        if (cw == 0 && lane < MT) red[20 + lane] = xs_bits;
         if (!csync()) break;
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
@@ -559,13 +633,15 @@ __global__ void __launch_bounds__(ChainCfg<MT>::kThreads, ChainCfg<MT>::kCtasPer
         }
       }
       // The barrier orders every thread's stores and adds before thread 0's
-      // release: the count makes them visible at gpu scope (cumulatively).
+      // release: the counts make them visible at gpu scope (cumulatively).
+      // A row tile is complete when its count reaches `splits`; with one
+      // token the problem's done counter also counts the item.
       if (!csync()) break;
       if (ctid == 0) {
-        red_release_gpu_add(cp.done + P.idx * kChainDoneStride, 1);
-        if (!whole)
-          *last_flag = atom_acq_rel_gpu_add(cp.cnt_base + P.cnt + md.row0 / kGemvTileRows, 1) ==
-                       P.splits - 1;
+        int32_t* tc = cp.cnt_base + P.cnt + md.row0 / kGemvTileRows;
+        if (MT == 1) red_release_gpu_add(cp.done + P.idx * kChainDoneStride, 1);
+        if (!whole) *last_flag = atom_acq_rel_gpu_add(tc, 1) == P.splits - 1;
+        else if (MT != 1) red_release_gpu_add(tc, 1);
       }
       if (!whole) {
         if (!csync()) break;
