@@ -86,6 +86,10 @@ def parse_args(argv=None):
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the gate 6912x2560 prefill GEMM at M=2048 (a small case "
                          "for profiling the tensor-core kernel) and print its own line")
+    ap.add_argument("--chain-only", action="store_true",
+                    help="time only the dependency-staged 30-layer step as one chain call at "
+                         "--batch tokens (1 or 2; a case for profiling the chain kernel) and "
+                         "print its own line")
     args = ap.parse_args(argv)
     if args.batch is None:
         args.batch = DEFAULT_BATCH[args.config]
@@ -1204,12 +1208,29 @@ def run_prefill_only(args):
     return 0
 
 
+def run_chain_only(args):
+    """The dependency-staged step (4 x layers stages) as one chain call:
+    `warmup` then `steps` graph replays, outputs checked against the same
+    stages run as separate batched calls."""
+    import torch
+
+    from i2_mpgemm_b200 import i2s, inputs
+    m = args.batch if args.batch in (1, 2) else 1
+    res = staged_chain_measurement(i2s, torch, inputs, args.layers, m, max(2, 2 * args.steps),
+                                   load_peaks())
+    res["workload"] = f"dependency-staged {args.layers}-layer step, one chain call, batch {m}"
+    print(json.dumps(res))
+    return 0 if res["matches_staged_calls"] else 1
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.prefill_only:
         return run_prefill_only(args)
+    if args.chain_only:
+        return run_chain_only(args)
     return run_native(args)
 
 
