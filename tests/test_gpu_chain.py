@@ -156,16 +156,33 @@ def test_chain_longer_than_one_launch(i2s):
     ch.check(ch.oracle(), "140 stages")
 
 
-def test_one_problem_and_wide_stage(i2s):
+@pytest.mark.parametrize("m", [1, 2])
+def test_one_problem_and_wide_stage(i2s, m):
     """A chain of one problem is the fused call; a stage wider than the grid
-    (more row tiles than CTAs) keeps one slice per problem."""
-    ch = Chain(i2s, [("one", 300, 640, "x")], [0], 1, 4100)
-    i2s.bitnet_i2s_quant_gemv_chain(ch.problems(), [0], 1)
+    (more row tiles than CTAs) keeps one slice per problem, and the next
+    problem reads a 64000-wide row (more than 32 of each warp's 512-chunks,
+    so the two-token path polls them in several rounds)."""
+    ch = Chain(i2s, [("one", 300, 640, "x")], [0], m, 4100)
+    i2s.bitnet_i2s_quant_gemv_chain(ch.problems(), [0], m)
     ch.check(ch.oracle(), "one")
     specs = [("wide", 128 * 500, 256, "x"), ("next", 256, 128 * 500, 0)]
-    ch = Chain(i2s, specs, [0, 1], 1, 4200)
-    i2s.bitnet_i2s_quant_gemv_chain(ch.problems(), [0, 1], 1)
+    ch = Chain(i2s, specs, [0, 1], m, 4200)
+    i2s.bitnet_i2s_quant_gemv_chain(ch.problems(), [0, 1], m)
     ch.check(ch.oracle(), "wide")
+
+
+@pytest.mark.parametrize("m", [1, 2])
+def test_stage_wider_than_the_grid_reads_chained_sources(i2s, m):
+    """Stage 1 has 1000 items (two 64000-row problems), more than the grid's
+    CTAs, so CTAs take several of its items and reuse the absmax of a source
+    they have already read: b's items (4 boxes each) read their slice again,
+    b2's (one box) keep it from the first pass."""
+    specs = [("a", 2048, 384, "x"), ("a2", 256, 384, "x"),
+             ("b", 128 * 500, 2048, 0), ("b2", 128 * 500, 256, 1)]
+    stages = [0, 0, 1, 1]
+    ch = Chain(i2s, specs, stages, m, 4300, acc=False)
+    i2s.bitnet_i2s_quant_gemv_chain(ch.problems(), stages, m)
+    ch.check(ch.oracle(), f"wide stage M={m}")
 
 
 def test_repeats_on_one_workspace_and_graph_replay(i2s):
