@@ -20,6 +20,7 @@
 #include "chain_kernel.cuh"
 #include "gemv_kernel.cuh"
 #include "mma_kernel.cuh"
+#include "prefill_kernel.cuh"
 #include "quant_kernels.cuh"
 
 namespace {
@@ -393,15 +394,41 @@ bitnet_status launch_mma_t(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStr
   return BITNET_OK;
 }
 
+// The prefill kernel: tiles of 128 tokens, both operands in shared memory.
+template <int CAP>
+bitnet_status launch_prefill(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
+                             bool pdl, bool wait, int dev) {
+  using C = PrefillCfg;
+  static std::atomic<uint8_t> smem_done[kMaxDevices];
+  auto kern = i2s_prefill_kernel<CAP>;
+  bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
+  if (st != BITNET_OK) return st;
+  if ((st = plan_mma<C::T>(bp, xq)) != BITNET_OK) return st;
+  bp.pdl = (pdl && wait) ? 1 : 0;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim =
+      dim3(static_cast<unsigned>(std::min(bp.total_items, C::kCtasPerSm * sm_count(dev))));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr = pdl_attr(pdl);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, bp);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the I2_S prefill kernel");
+  return BITNET_OK;
+}
+
 // Token tile by M: 16, 32 or 64 tokens for decode (3 or 4 CTAs per SM),
-// 128 for prefill (2 CTAs per SM).
+// the prefill kernel above 64 tokens.
 template <int CAP>
 bitnet_status launch_mma(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
                          bool pdl, bool wait, int dev) {
   if (bp.m <= 16) return launch_mma_t<16>(bp, xq, stream, pdl, wait, dev);
   if (bp.m <= 32) return launch_mma_t<32>(bp, xq, stream, pdl, wait, dev);
   if (bp.m <= 64) return launch_mma_t<64>(bp, xq, stream, pdl, wait, dev);
-  return launch_mma_t<128>(bp, xq, stream, pdl, wait, dev);
+  return launch_prefill(bp, xq, stream, pdl, wait, dev);
 }
 
 MmaProblem make_mma_problem(const uint8_t* packed, int64_t n, int64_t k, const float* xs, float* y,
