@@ -394,13 +394,13 @@ bitnet_status launch_mma_t(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStr
   return BITNET_OK;
 }
 
-// The prefill kernel: tiles of 128 tokens, both operands in shared memory.
-template <int CAP>
+// The prefill kernel: tiles of T tokens, both operands in shared memory.
+template <int T, int CAP>
 bitnet_status launch_prefill(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
                              bool pdl, bool wait, int dev) {
-  using C = PrefillCfg;
+  using C = PrefillCfg<T>;
   static std::atomic<uint8_t> smem_done[kMaxDevices];
-  auto kern = i2s_prefill_kernel<CAP>;
+  auto kern = i2s_prefill_kernel<T, CAP>;
   bitnet_status st = ensure_smem(kern, C::kSmemBytes, dev, smem_done);
   if (st != BITNET_OK) return st;
   if ((st = plan_mma<C::T>(bp, xq)) != BITNET_OK) return st;
@@ -420,15 +420,18 @@ bitnet_status launch_prefill(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaS
   return BITNET_OK;
 }
 
-// Token tile by M: 16, 32 or 64 tokens for decode (3 or 4 CTAs per SM),
-// the prefill kernel above 64 tokens.
+// Token tile by M, as measured best: 16 or 32 tokens on the TMEM-A kernel
+// (4 CTAs per SM); 64 tokens on the shared-memory kernel (large layer at
+// M = 64: 1.52 TB/s against 1.25 on the TMEM-A kernel at 64 tokens); 128
+// tokens above (64-token tiles there lose more to unpacking per MAC than
+// they gain in tiles: gate 6912x2560 at M = 512, 0.56 against 0.68 POPS).
 template <int CAP>
 bitnet_status launch_mma(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
                          bool pdl, bool wait, int dev) {
   if (bp.m <= 16) return launch_mma_t<16>(bp, xq, stream, pdl, wait, dev);
   if (bp.m <= 32) return launch_mma_t<32>(bp, xq, stream, pdl, wait, dev);
-  if (bp.m <= 64) return launch_mma_t<64>(bp, xq, stream, pdl, wait, dev);
-  return launch_prefill(bp, xq, stream, pdl, wait, dev);
+  if (bp.m <= 64) return launch_prefill<64>(bp, xq, stream, pdl, wait, dev);
+  return launch_prefill<128>(bp, xq, stream, pdl, wait, dev);
 }
 
 MmaProblem make_mma_problem(const uint8_t* packed, int64_t n, int64_t k, const float* xs, float* y,

@@ -1,12 +1,14 @@
-// prefill_kernel.cuh -- the I2_S ternary x int8 matmul at prefill sizes
-// (more than 64 tokens) on the sm_100a tensor cores, with both MMA operands
-// in shared memory and two accumulator buffers in tensor memory.
+// prefill_kernel.cuh -- the I2_S ternary x int8 matmul at 33 tokens and
+// more (64-token tiles up to 64 tokens, 128-token tiles above) on the
+// sm_100a tensor cores, with both MMA operands in shared memory and two
+// accumulator buffers in tensor memory.
 //
 // Same contraction, tile and correction as the decode-sized tensor kernel
 // (mma_kernel.cuh): swap-AB, MMA M = 128 rows of unsigned codes c = w + 1
 // with row 127 all ones (so D[127] = sum_k x and acc = D[r] - D[127]), MMA
-// N = 128 tokens of Xq, one 127 x 128 output tile over the whole K per work
-// item.  What differs is where the unpacked weights go.  There, they are
+// N = T tokens of Xq, one 127 x T output tile over the whole K per work
+// item (T = 64 or 128 tokens).  What differs is where the unpacked weights
+// go.  There, they are
 // stored into tensor memory, which then has no room for a second
 // accumulator, so the epilogue of a tile (tensor memory -> fp32 outputs)
 // and the next tile's MMAs take turns.  Here the unpack warps write each
@@ -23,7 +25,7 @@
 //
 // Roles (10 warps):
 //   warp 0     TMA producer: packed weights (a 128-row x 128-byte box, four
-//              I2_S blocks, per stage) and Xq (a 128-token x 128-byte box
+//              I2_S blocks, per stage) and Xq (a T-token x 128-byte box
 //              per block), both with the 128-byte swizzle.
 //   warp 1     tensor-memory allocator and MMA issuer (one thread).
 //   warps 2-5  unpack: thread r owns weight row r; per block it writes its
@@ -43,19 +45,20 @@
 
 namespace bitnet {
 
-// CTAS CTAs per SM; WSTAGES weight boxes, XSTAGES activation boxes and
-// ASLOTS A slots per CTA.
-template <int CTAS, int WSTAGES, int XSTAGES, int ASLOTS>
+// TOKENS per tile (MMA N); CTAS CTAs per SM; WSTAGES weight boxes,
+// XSTAGES activation boxes and ASLOTS A slots per CTA.
+template <int TOKENS, int CTAS, int WSTAGES, int XSTAGES, int ASLOTS>
 struct PrefillCfgT {
-  static constexpr int T = 128;               // tokens per tile (MMA N)
+  static_assert(TOKENS == 64 || TOKENS == 128, "token tile");
+  static constexpr int T = TOKENS;            // tokens per tile (MMA N)
   static constexpr int kThreads = 320;        // 10 warps
   static constexpr int kCtasPerSm = CTAS;
   static constexpr int kDBufs = 2;            // accumulator buffers
-  static constexpr uint32_t kDCols = 128;     // columns of one buffer
-  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kDCols = T;       // columns of one buffer
+  static constexpr uint32_t kTmemCols = pow2_at_least(2 * T);
   static constexpr int kWBytes = 128 * 128;   // weight box: 128 rows x 128 B
   static constexpr int kWStages = WSTAGES;
-  static constexpr int kXBox = T * 128;       // activation box: 128 tokens x 128 B
+  static constexpr int kXBox = T * 128;       // activation box: T tokens x 128 B
   static constexpr int kXStages = XSTAGES;
   static constexpr int kABytes = 128 * 128;   // one block of codes: 128 rows x 128 B
   static constexpr int kASlots = ASLOTS;
@@ -69,12 +72,14 @@ struct PrefillCfgT {
   static_assert((kSmemBytes + 1024) * kCtasPerSm <= 228 * 1024, "shared memory per SM");
 };
 
-// Measured on the B200 (gate 6912x2560 / down 2560x6912 at M = 2048):
-// 2 CTAs with 1 weight stage, 3 activation stages and 2 A slots, 1.21 / 0.95
-// POPS; 2 CTAs with 2 / 2 / 2, 1.20 / 0.93; 2 CTAs with 1 / 2 / 3, 1.22 /
-// 0.93; 1 CTA with 2 / 6 / 4, 0.97 / 0.91.  Shared memory allows no deeper
-// rings at 2 CTAs per SM.
-using PrefillCfg = PrefillCfgT<2, 1, 3, 2>;
+// Measured on the B200 (gate 6912x2560 / down 2560x6912 at M = 2048, T =
+// 128): 2 CTAs with 1 weight stage, 3 activation stages and 2 A slots, 1.21
+// / 0.95 POPS; 2 CTAs with 2 / 2 / 2, 1.20 / 0.93; 2 CTAs with 1 / 2 / 3,
+// 1.22 / 0.93; 1 CTA with 2 / 6 / 4, 0.97 / 0.91.  Shared memory allows no
+// deeper rings at 2 CTAs per SM.  At T = 64 the activation boxes are half
+// the size: 4 stages and 3 A slots.
+template <int T>
+using PrefillCfg = PrefillCfgT<T, 2, 1, (T == 128 ? 3 : 4), (T == 128 ? 2 : 3)>;
 
 // Make this thread's generic-proxy shared-memory writes visible to the
 // tensor core (async proxy).
@@ -93,10 +98,10 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-template <int CAP>
-__global__ void __launch_bounds__(PrefillCfg::kThreads, PrefillCfg::kCtasPerSm)
+template <int TOK, int CAP>
+__global__ void __launch_bounds__(PrefillCfg<TOK>::kThreads, PrefillCfg<TOK>::kCtasPerSm)
     i2s_prefill_kernel(const __grid_constant__ MmaParamsT<CAP> bp) {
-  using C = PrefillCfg;
+  using C = PrefillCfg<TOK>;
   constexpr int T = C::T;
   constexpr int WS = C::kWStages, XS = C::kXStages, AS = C::kASlots, DB = C::kDBufs;
 
