@@ -1109,7 +1109,10 @@ def run_native(args):
                     "peak_source": peaks["source"],
                     "kernel": ("i2s_gemv_dp4a_kernel (persistent launches of up to 160 problems)"
                                if dp4a else
-                               "i2s_mma_kernel (persistent launches of up to 96 problems)"),
+                               ("i2s_mma_kernel (persistent launches of up to 96 problems)"
+                                if m <= 32 else
+                                "i2s_prefill_kernel, 64-token tiles (persistent launches of up "
+                                "to 96 problems)")),
                     "launches_per_step": k_launches,
                     "bytes_per_launch": int(k_bytes // k_launches),
                     "launch_us_mean": round(1000 * k_ms / k_launches, 3)}
@@ -1120,7 +1123,9 @@ def run_native(args):
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_tops, 1),
                     "unit": "TOPS", "frac": round(achieved / int8_tops, 4), "traffic": None,
                     "peak_source": int8_src,
-                    "kernel": "i2s_mma_kernel (persistent tcgen05 kind::i8)",
+                    "kernel": ("i2s_prefill_kernel (persistent tcgen05 kind::i8, both operands "
+                               "in shared memory)" if m > 32 else
+                               "i2s_mma_kernel (persistent tcgen05 kind::i8)"),
                     "launches_per_step": k_launches,
                     "ops_per_launch": int(work.work // k_launches),
                     "launch_us_mean": round(1000 * k_ms / k_launches, 3)}
