@@ -275,6 +275,25 @@ def test_prefill_shapes_sampled(i2s, m):
         _check_sampled(i2s, packed, d_packed, n, k, x, t, 2048, seed, f"{name} M={m}")
 
 
+def test_prefill_gate_in_full(i2s):
+    """gate 6912x2560 at M = 2048, every output: the int32 accumulators
+    against an exact product of the generator's ternary matrix with the
+    oracle's int8 codes (float64 BLAS; every sum is below 2^53, so exact),
+    and each fp32 output against ((float)acc * xs) * s in that order."""
+    n, k, m = 6912, 2560, 2048
+    seed = inputs.seed_prefill(0)
+    w, t, s = inputs.ternary_weights(n, k, seed)
+    x = inputs.activations(m, k, seed)
+    packed, d_packed = _packed_pair(i2s, w)
+    y, acc = i2s.bitnet_i2s_quant_gemv(d_packed, n, k, dev(x), want_acc=True)
+    xq, xs = oracle.act_quant(x.numpy())
+    want = (xq.astype(np.float64) @ t.numpy().astype(np.float64).T).astype(np.int64)
+    assert_acc_equal(acc.cpu().numpy(), want.astype(np.int32), "gate M=2048")
+    scale = np.float32(oracle.scale(packed, n, k))
+    y_ref = (want.astype(np.float32) * xs[:, None]).astype(np.float32) * scale
+    assert_y_close(y.cpu().numpy(), y_ref.astype(np.float32), "gate M=2048")
+
+
 @pytest.mark.parametrize("m", [1, 64])
 def test_large_layer_sampled(i2s, m):
     for idx, p in enumerate(inputs.projections_large()):
