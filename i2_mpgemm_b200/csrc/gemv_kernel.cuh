@@ -353,7 +353,14 @@ __global__ void __launch_bounds__(GemvCfg<MT, KMAX>::kThreads, GemvCfg<MT, KMAX>
           ++item;
         } else if (dyn) {
           if (!have_next) {
-            if (!waited) wait_for_inputs();
+            if (!waited) {
+              // Activations whose loads waited for the preceding grid go
+              // out now: the next box may need a stage that the compute
+              // warps free only once they have them.
+              wait_for_inputs();
+              load_pending_x();
+              if (!ok) break;
+            }
             grab();
           }
           item = next;
