@@ -152,6 +152,12 @@ def step_launches(m: int, ks) -> int:
     return -(-len(ks) // 1000) + -(-small // DECODE_BATCH) + -(-(len(ks) - small) // MMA_BATCH)
 
 
+def prefill_tile(m: int) -> int:
+    """Token tile of the shared-memory tensor kernel at M tokens (the library
+    routes 33-64 tokens to 64-token tiles, up to 1024 to 128, above to 256)."""
+    return 64 if m <= 64 else (128 if m <= 1024 else 256)
+
+
 def code_digest(paths) -> str:
     """sha256 of the code of the given sources with comments and blank lines
     removed, so that a comment edit keeps a capture valid and a code edit
@@ -1128,9 +1134,9 @@ def run_native(args):
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_tops, 1),
                     "unit": "TOPS", "frac": round(achieved / int8_tops, 4), "traffic": None,
                     "peak_source": int8_src,
-                    "kernel": ("i2s_prefill_kernel (persistent tcgen05 kind::i8, both operands "
-                               "in shared memory)" if m > 32 else
-                               "i2s_mma_kernel (persistent tcgen05 kind::i8)"),
+                    "kernel": ((f"i2s_prefill_kernel, {prefill_tile(m)}-token tiles "
+                                "(persistent tcgen05 kind::i8, both operands in shared memory)")
+                               if m > 32 else "i2s_mma_kernel (persistent tcgen05 kind::i8)"),
                     "launches_per_step": k_launches,
                     "ops_per_launch": int(work.work // k_launches),
                     "launch_us_mean": round(1000 * k_ms / k_launches, 3)}

@@ -423,15 +423,19 @@ bitnet_status launch_prefill(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaS
 // Token tile by M, as measured best: 16 or 32 tokens on the TMEM-A kernel
 // (4 CTAs per SM); 64 tokens on the shared-memory kernel (large layer at
 // M = 64: 1.52 TB/s against 1.25 on the TMEM-A kernel at 64 tokens); 128
-// tokens above (64-token tiles there lose more to unpacking per MAC than
-// they gain in tiles: gate 6912x2560 at M = 512, 0.56 against 0.68 POPS).
+// tokens up to M = 1024 (64-token tiles there lose more to unpacking per MAC
+// than they gain in tiles: gate 6912x2560 at M = 512, 0.56 against 0.68
+// POPS); 256 tokens above, one CTA per SM (gate + up + down 6912x2560 /
+// 2560x6912 at M = 2048: 160 against 166 us per set; at M = 1024 the two
+// tie, at M = 512 the 128-token tile is 8 % faster).
 template <int CAP>
 bitnet_status launch_mma(MmaParamsT<CAP>& bp, const int8_t* const* xq, cudaStream_t stream,
                          bool pdl, bool wait, int dev) {
   if (bp.m <= 16) return launch_mma_t<16>(bp, xq, stream, pdl, wait, dev);
   if (bp.m <= 32) return launch_mma_t<32>(bp, xq, stream, pdl, wait, dev);
   if (bp.m <= 64) return launch_prefill<64>(bp, xq, stream, pdl, wait, dev);
-  return launch_prefill<128>(bp, xq, stream, pdl, wait, dev);
+  if (bp.m <= 1024) return launch_prefill<128>(bp, xq, stream, pdl, wait, dev);
+  return launch_prefill<256>(bp, xq, stream, pdl, wait, dev);
 }
 
 MmaProblem make_mma_problem(const uint8_t* packed, int64_t n, int64_t k, const float* xs, float* y,

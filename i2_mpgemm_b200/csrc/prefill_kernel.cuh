@@ -1,5 +1,6 @@
 // prefill_kernel.cuh -- the I2_S ternary x int8 matmul at 33 tokens and
-// more (64-token tiles up to 64 tokens, 128-token tiles above) on the
+// more (64-token tiles up to 64 tokens, 128-token tiles up to 1024, 256-token
+// tiles above) on the
 // sm_100a tensor cores, with both MMA operands in shared memory and two
 // accumulator buffers in tensor memory.
 //
@@ -7,7 +8,7 @@
 // (mma_kernel.cuh): swap-AB, MMA M = 128 rows of unsigned codes c = w + 1
 // with row 127 all ones (so D[127] = sum_k x and acc = D[r] - D[127]), MMA
 // N = T tokens of Xq, one 127 x T output tile over the whole K per work
-// item (T = 64 or 128 tokens).  What differs is where the unpacked weights
+// item (T = 64, 128 or 256 tokens).  What differs is where the unpacked weights
 // go.  There, they are
 // stored into tensor memory, which then has no room for a second
 // accumulator, so the epilogue of a tile (tensor memory -> fp32 outputs)
@@ -33,11 +34,14 @@
 //              makes them visible to the tensor core (proxy fence).
 //   warps 6-9  epilogue: each reads the accumulator lanes of its quarter and
 //              writes y = ((float)acc * xs[m]) * s, token-major; the token
-//              sums of row 127 reach the others through shared memory.
+//              sums of row 127 and the tile's token scales (fetched from
+//              global memory while the accumulator fills) reach the others
+//              through shared memory.
 //
 // Barriers: fullw/emptyw (weight ring), fullx/emptyx (activation ring),
 // afull/aempty (A slots: unpack -> MMA -> unpack), dfull/dempty
-// (accumulators: MMA -> epilogue -> MMA), xsum (row 127's token sums).
+// (accumulators: MMA -> epilogue -> MMA), xsum (row 127's token sums and the
+// tile's token scales, written to shared memory by the epilogue warps).
 // Every wait is bounded (ptx.cuh).
 #pragma once
 
@@ -49,7 +53,7 @@ namespace bitnet {
 // XSTAGES activation boxes and ASLOTS A slots per CTA.
 template <int TOKENS, int CTAS, int WSTAGES, int XSTAGES, int ASLOTS>
 struct PrefillCfgT {
-  static_assert(TOKENS == 64 || TOKENS == 128, "token tile");
+  static_assert(TOKENS == 64 || TOKENS == 128 || TOKENS == 256, "token tile");
   static constexpr int T = TOKENS;            // tokens per tile (MMA N)
   static constexpr int kThreads = 320;        // 10 warps
   static constexpr int kCtasPerSm = CTAS;
@@ -63,23 +67,30 @@ struct PrefillCfgT {
   static constexpr int kABytes = 128 * 128;   // one block of codes: 128 rows x 128 B
   static constexpr int kASlots = ASLOTS;
   static constexpr int kNumBars = 2 * kWStages + 2 * kXStages + 2 * kASlots + 2 * kDBufs + 2;
+  // Rings, barriers (an even count: the arrays after them stay 16-byte
+  // aligned), then per accumulator buffer the token sums and token scales.
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kWStages) * kWBytes +
                                        static_cast<size_t>(kXStages) * kXBox +
                                        static_cast<size_t>(kASlots) * kABytes + kNumBars * 8 +
-                                       2 * T * 4 + 16;
+                                       2 * T * 4 + 2 * T * 4 + 16;
   static constexpr uint32_t kIdesc = idesc_i8(128, T, false, true);  // u8 codes x s8
   static_assert(kTmemCols * kCtasPerSm <= 512, "tensor memory per SM");
   static_assert((kSmemBytes + 1024) * kCtasPerSm <= 228 * 1024, "shared memory per SM");
 };
 
 // Measured on the B200 (gate 6912x2560 / down 2560x6912 at M = 2048, T =
-// 128): 2 CTAs with 1 weight stage, 3 activation stages and 2 A slots, 1.21
-// / 0.95 POPS; 2 CTAs with 2 / 2 / 2, 1.20 / 0.93; 2 CTAs with 1 / 2 / 3,
-// 1.22 / 0.93; 1 CTA with 2 / 6 / 4, 0.97 / 0.91.  Shared memory allows no
-// deeper rings at 2 CTAs per SM.  At T = 64 the activation boxes are half
-// the size: 4 stages and 3 A slots.
+// 128, with an earlier epilogue that fetched token scales per 16 columns):
+// 2 CTAs with 1 weight stage, 3 activation stages and 2 A slots, 1.21 / 0.95
+// POPS; 2 CTAs with 2 / 2 / 2, 1.20 / 0.93; 2 CTAs with 1 / 2 / 3, 1.22 /
+// 0.93; 1 CTA with 2 / 6 / 4, 0.97 / 0.91.  Shared memory allows no deeper
+// rings at 2 CTAs per SM.  At T = 64 the activation boxes are half the size:
+// 4 stages and 3 A slots.  At T = 256 the two accumulators fill tensor
+// memory, so one CTA runs per SM: 2 weight stages, 4 activation boxes of 32
+// KB and 3 A slots (218 KB of shared memory); the splits 1/4/4, 2/3/5,
+// 1/5/2, 1/3/6 and two 128-token boxes per stage were within 3 % of it.
 template <int T>
-using PrefillCfg = PrefillCfgT<T, 2, 1, (T == 128 ? 3 : 4), (T == 128 ? 2 : 3)>;
+using PrefillCfg = PrefillCfgT<T, (T == 256 ? 1 : 2), (T == 256 ? 2 : 1),
+                               (T == 128 ? 3 : 4), (T == 128 ? 2 : 3)>;
 
 // Make this thread's generic-proxy shared-memory writes visible to the
 // tensor core (async proxy).
@@ -113,7 +124,8 @@ __global__ void __launch_bounds__(PrefillCfg<TOK>::kThreads, PrefillCfg<TOK>::kC
   uint8_t* aring = xring + XS * C::kXBox;
   uint64_t* bars = reinterpret_cast<uint64_t*>(aring + AS * C::kABytes);
   int32_t* xsum_smem = reinterpret_cast<int32_t*>(bars + C::kNumBars);  // [2][T]
-  uint32_t* misc = reinterpret_cast<uint32_t*>(xsum_smem + 2 * T);     // [0] tmem, [1] abort
+  float* xs_smem = reinterpret_cast<float*>(xsum_smem + 2 * T);          // [2][T]
+  uint32_t* misc = reinterpret_cast<uint32_t*>(xs_smem + 2 * T);         // [0] tmem, [1] abort
   volatile uint32_t* abort_flag = misc + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -148,8 +160,8 @@ __global__ void __launch_bounds__(PrefillCfg<TOK>::kThreads, PrefillCfg<TOK>::kC
       mbar_init(dfull_bar(b), 1);   // MMA commit
       mbar_init(dempty_bar(b), 4);  // the four epilogue warps
     }
-    mbar_init(xsum_bar(0), 1);  // row 127's thread
-    mbar_init(xsum_bar(1), 1);
+    mbar_init(xsum_bar(0), 4);  // the four epilogue warps
+    mbar_init(xsum_bar(1), 4);
     misc[1] = 0u;
     fence_mbar_init();
   }
@@ -357,6 +369,7 @@ __global__ void __launch_bounds__(PrefillCfg<TOK>::kThreads, PrefillCfg<TOK>::kC
     const int quarter = warp & 3;  // tensor-memory lanes this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    constexpr int kXsPer = (T + 127) / 128;  // token scales each thread fetches
     bool ok = true;
     int ii = 0;
     for (int item = item_lo; item < item_hi && ok; ++item, ++ii) {
@@ -364,53 +377,78 @@ __global__ void __launch_bounds__(PrefillCfg<TOK>::kThreads, PrefillCfg<TOK>::kC
       mma_item(bp, item, &p, &rt, &tt);
       const MmaProblem& P = bp.p[p];
       const int b = ii % DB;
+      const int64_t tok0 = static_cast<int64_t>(tt) * T;
+      // The tile's token scales are fetched while its accumulator fills:
+      // thread r takes tokens r and r + 128.
+      float xsr[kXsPer];
+#pragma unroll
+      for (int i = 0; i < kXsPer; ++i) {
+        const int j = r + 128 * i;
+        xsr[i] = (j < T && tok0 + j < m_tokens) ? __ldg(P.xs + tok0 + j) : 0.0f;
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(dfull_bar(b), (ii / DB) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      // Both arrays of this buffer parity were last read for item ii - 2,
+      // which every epilogue warp finished before the accumulator of item
+      // ii could be filled.
       int32_t* xsum_buf = xsum_smem + (ii & 1) * T;
+      float* xs_buf = xs_smem + (ii & 1) * T;
+#pragma unroll
+      for (int i = 0; i < kXsPer; ++i) {
+        const int j = r + 128 * i;
+        if (j < T) xs_buf[j] = xsr[i];
+      }
       if (quarter == 3) {
         // Row 127 (this warp's lane 31) holds sum_k x of every token.
 #pragma unroll 1
-        for (int c0 = 0; c0 < T; c0 += 16) {
-          uint32_t v[16];
+        for (int c0 = 0; c0 < T; c0 += 32) {
+          uint32_t v[16], w[16];
           tmem_ld_32x32b_x16(tmem + lane_base + b * C::kDCols + c0, v);
+          tmem_ld_32x32b_x16(tmem + lane_base + b * C::kDCols + c0 + 16, w);
           tmem_ld_wait();
           if (lane == 31) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xsum_buf[c0 + j] = static_cast<int32_t>(v[j]);
+            for (int j = 0; j < 16; ++j) {
+              xsum_buf[c0 + j] = static_cast<int32_t>(v[j]);
+              xsum_buf[c0 + 16 + j] = static_cast<int32_t>(w[j]);
+            }
           }
         }
-        if (lane == 31) mbar_arrive(xsum_bar(ii & 1));
-        __syncwarp();
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xsum_bar(ii & 1));
       ok = __all_sync(0xffffffffu, mbar_wait(xsum_bar(ii & 1), (ii >> 1) & 1, abort_flag));
       if (!ok) break;
       const float s = *reinterpret_cast<const float*>(P.packed + static_cast<int64_t>(P.n) * (P.k >> 2));
       const int64_t n = static_cast<int64_t>(rt) * kMmaTileRows + r;
-      const int64_t tok0 = static_cast<int64_t>(tt) * T;
       const int64_t nn = P.n;
       const bool row_ok = r < kMmaTileRows && n < nn;
       float* __restrict__ yb = P.y;
       int32_t* __restrict__ ab = P.acc;
-      const float* __restrict__ xsb = P.xs;
 #pragma unroll 1
-      for (int c0 = 0; c0 < T; c0 += 16) {
+      for (int c0 = 0; c0 < T; c0 += 32) {
         if (tok0 + c0 >= m_tokens) break;  // warp-uniform
-        float xsv[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          xsv[j] = (tok0 + c0 + j < m_tokens) ? __ldg(xsb + tok0 + c0 + j) : 0.0f;
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem + lane_base + b * C::kDCols + c0, v);
+        uint32_t v0[16], v1[16];
+        tmem_ld_32x32b_x16(tmem + lane_base + b * C::kDCols + c0, v0);
+        tmem_ld_32x32b_x16(tmem + lane_base + b * C::kDCols + c0 + 16, v1);
         tmem_ld_wait();
         if (row_ok) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int64_t tok = tok0 + c0 + j;
-            if (tok < m_tokens) {
-              const int32_t a = static_cast<int32_t>(v[j]) - xsum_buf[c0 + j];
-              yb[tok * nn + n] = __fmul_rn(__fmul_rn(__int2float_rn(a), xsv[j]), s);
-              if (ab != nullptr) ab[tok * nn + n] = a;
+          for (int g = 0; g < 8; ++g) {
+            const int4 sums = *reinterpret_cast<const int4*>(xsum_buf + c0 + 4 * g);
+            const float4 scl = *reinterpret_cast<const float4*>(xs_buf + c0 + 4 * g);
+            const int32_t sm[4] = {sums.x, sums.y, sums.z, sums.w};
+            const float sc[4] = {scl.x, scl.y, scl.z, scl.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 4 * g + e;
+              const int64_t tok = tok0 + c0 + j;
+              if (tok < m_tokens) {
+                const int32_t a = static_cast<int32_t>(j < 16 ? v0[j] : v1[j - 16]) - sm[e];
+                yb[tok * nn + n] = __fmul_rn(__fmul_rn(__int2float_rn(a), sc[e]), s);
+                if (ab != nullptr) ab[tok * nn + n] = a;
+              }
             }
           }
         }

@@ -94,14 +94,16 @@ def test_act_quant_worked_examples_and_zero_rows(i2s):
 # ------------------------------------------------------------- matmul, full
 
 # (M, N, K): several 128-row tiles with ragged N, every token tile size with
-# ragged M, and K with a partial last 512-wide stage.
+# ragged M (past 128 and past 1024 tokens: several 128- or 256-token tiles,
+# the last one ragged), and K with a partial last 512-wide stage.
 # The tensor-core tile has 127 weight rows (TMEM lane 127 carries the token
 # sums), so 127, 128, 254 and 255 rows sit on and next to tile edges; 128 and
 # 255 also sit on the decode kernel's.
 SMALL = [(1, 1, 128), (1, 7, 640), (3, 130, 384), (16, 300, 1152), (17, 129, 640),
          (33, 257, 512), (64, 200, 1024), (65, 131, 640), (130, 300, 896), (200, 64, 256),
          (5, 127, 256), (9, 124, 384), (20, 128, 384), (70, 254, 640), (3, 255, 128),
-         (129, 381, 512)]
+         (129, 381, 512), (256, 127, 256), (300, 200, 640), (513, 131, 384),
+         (1100, 131, 384), (1025, 254, 640)]
 
 
 def _case(m, n, k, seed):
