@@ -1,6 +1,7 @@
 """Host-side logic of bench.py, without a GPU: the launch count it reports,
-the workload description it prints, and the rule that ties the recorded
-DRAM traffic to the kernel code it was captured on."""
+the workload description it prints, the rule that ties the recorded
+DRAM traffic to the kernel code it was captured on, and the warm-up of a
+rotation of graphs."""
 import importlib.util
 import os
 
@@ -95,3 +96,53 @@ def test_reference_arm_line_on_a_small_sample(bench, capsys):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["config"] == bench.workload_config(0, 1, 30, 1)
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+class _FakeCuda:
+    """Records graph replays and event records in order (no GPU)."""
+
+    def __init__(self, log):
+        self.log = log
+
+    def synchronize(self):
+        pass
+
+    def Event(self, enable_timing=False):
+        log = self.log
+
+        class _Ev:
+            def record(self):
+                log.append(("record",))
+
+            def synchronize(self):
+                pass
+
+            def elapsed_time(self, other):
+                return 1.0
+
+        return _Ev()
+
+
+class _FakeGraph:
+    def __init__(self, log, idx):
+        self.log, self.idx = log, idx
+
+    def replay(self):
+        self.log.append(("replay", self.idx))
+
+
+def test_rotation_replays_every_graph_before_the_timed_region(bench):
+    """A graph's first replay uploads it; with a rotation longer than the
+    warm-up, every graph must still have been replayed once before the start
+    event, and the timed region must replay exactly `steps` graphs."""
+    import types
+    log = []
+    torch = types.SimpleNamespace(cuda=_FakeCuda(log))
+    graphs = [_FakeGraph(log, i) for i in range(16)]
+    ms = bench.time_replays(torch, graphs, steps=20, warmup=5, collective=False)
+    start = log.index(("record",))
+    before = {e[1] for e in log[:start] if e[0] == "replay"}
+    assert before == set(range(16))
+    timed = [e for e in log[start + 1:] if e[0] == "replay"]
+    assert len(timed) == 20 and log[-1] == ("record",)
+    assert ms == pytest.approx(1.0 / 20)
