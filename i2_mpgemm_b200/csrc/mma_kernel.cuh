@@ -38,9 +38,10 @@
 //
 // The MMA-issuing thread spends tens of cycles per small MMA, so a decode
 // tile keeps the tensor pipe fed only with several issuers per SM: small
-// token tiles run 3 or 4 CTAs per SM (TMEM 128 columns each).  Above 64
-// tokens the library uses prefill_kernel.cuh instead (operands in shared
-// memory, two accumulators); the 128-token configuration here remains valid.
+// token tiles run 3 or 4 CTAs per SM (TMEM 128 columns each).  From 33
+// tokens on the library uses prefill_kernel.cuh instead (operands in shared
+// memory, two accumulators); the 64- and 128-token configurations here
+// remain valid.
 //
 // Unpack: the 32-bit word made of bytes 4i..4i+3 of a block, shifted right
 // by 6-2g and masked with 0x03030303, is the four codes of weights
