@@ -1,18 +1,17 @@
 // prefill_kernel.cuh -- the I2_S ternary x int8 matmul at 33 tokens and
 // more (64-token tiles up to 64 tokens, 128-token tiles up to 1024, 256-token
-// tiles above) on the
-// sm_100a tensor cores, with both MMA operands in shared memory and two
-// accumulator buffers in tensor memory.
+// tiles above) on the sm_100a tensor cores, with both MMA operands in shared
+// memory and two accumulator buffers in tensor memory.
 //
 // Same contraction, tile and correction as the decode-sized tensor kernel
 // (mma_kernel.cuh): swap-AB, MMA M = 128 rows of unsigned codes c = w + 1
 // with row 127 all ones (so D[127] = sum_k x and acc = D[r] - D[127]), MMA
 // N = T tokens of Xq, one 127 x T output tile over the whole K per work
-// item (T = 64, 128 or 256 tokens).  What differs is where the unpacked weights
-// go.  There, they are
-// stored into tensor memory, which then has no room for a second
-// accumulator, so the epilogue of a tile (tensor memory -> fp32 outputs)
-// and the next tile's MMAs take turns.  Here the unpack warps write each
+// item (T = 64, 128 or 256 tokens).  What differs is where the unpacked
+// weights go.  There, they are stored into tensor memory, which then has no
+// room for a second accumulator, so the epilogue of a tile (tensor memory
+// -> fp32 outputs) and the next tile's MMAs take turns.  Here the unpack
+// warps write each
 // 128 x 128-byte block of codes into shared memory in the layout the
 // 128-byte-swizzled TMA boxes of Xq have (rows of 128 bytes, 16-byte chunk c
 // of row r at c ^ (r % 8), 8-row groups 1024 bytes apart), and the MMA reads
@@ -21,8 +20,9 @@
 // contraction as a dense int8 product; "How BitNet's 1-Bit (I2_S)
 // Quantization Works Compared to Standard LLM Quantization", How I2_S
 // Kernels Process the Format: unpack once, reuse over many activations).
-// Tensor memory then holds two 128-column accumulators per CTA, and a
-// separate group of epilogue warps drains one while the MMAs fill the other.
+// Tensor memory then holds two T-column accumulators per CTA (at T = 256
+// they take all 512 columns, so one CTA runs per SM), and a separate group
+// of epilogue warps drains one while the MMAs fill the other.
 //
 // Roles (10 warps):
 //   warp 0     TMA producer: packed weights (a 128-row x 128-byte box, four
