@@ -11,11 +11,10 @@
 // weights go.  There, they are stored into tensor memory, which then has no
 // room for a second accumulator, so the epilogue of a tile (tensor memory
 // -> fp32 outputs) and the next tile's MMAs take turns.  Here the unpack
-// warps write each
-// 128 x 128-byte block of codes into shared memory in the layout the
-// 128-byte-swizzled TMA boxes of Xq have (rows of 128 bytes, 16-byte chunk c
-// of row r at c ^ (r % 8), 8-row groups 1024 bytes apart), and the MMA reads
-// both operands through shared-memory descriptors ("LLM Quantization
+// warps write each 128 x 128-byte block of codes into shared memory in the
+// layout the 128-byte-swizzled TMA boxes of Xq have (rows of 128 bytes,
+// 16-byte chunk c of row r at c ^ (r % 8), 8-row groups 1024 bytes apart),
+// and the MMA reads both operands through shared-memory descriptors ("LLM Quantization
 // Paradigms: FP8, AWQ, EXL2 & BitNet b1.58 in 2026", section 5: the ternary
 // contraction as a dense int8 product; "How BitNet's 1-Bit (I2_S)
 // Quantization Works Compared to Standard LLM Quantization", How I2_S
